@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark of the fused 4-bit codebook GEMV / GEMM on B200.
+
+A step is one Llama-2-7B decoder layer's four linears at M = 1 through
+q4_gemv (qkv 4096->12288, o 4096->4096, gate_up 4096->22016, down
+11008->4096), weights quantized from seeded N(0, 0.02) by q4_pack.  Eight
+distinct copies of the layer's packed weights (862 MB, several times the
+126 MB L2) rotate from step to step, so every step streams its weights from
+HBM.  The timed region replays CUDA graphs of these launches.
+
+The JSON line reports:
+  value         algorithmic GB/s = (code + scale + x + y + codebook bytes) per
+                step / device time per step, summed over ranks
+  roofline      the gate_up launch (largest share of the step), its algorithmic
+                bytes / its mean CUDA-event duration, against the measured HBM peak
+  e2e           the same metric through the Python API per step, with x copied
+                from pinned host memory and y read back every step
+  cpu_baseline  the oracle (single-threaded C) on the same layer, on the host
+  gemm_prefill  q4_gemm at M = 256 on the Llama-2-70B linears: TFLOP/s
+
+``--impl reference`` times the oracle instead (the reference arm).
+Multi-GPU (torchrun): independent replicas, one per rank (weak scaling); the
+timed region is bracketed by barriers and the max over ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+COPIES = 8
+GROUP = 64
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def algo_bytes(M, N, K):
+    """Algorithmic bytes of one q4 matmul: codes + scales + x + y + codebook."""
+    return N * K // 2 + N * (K // GROUP) * 2 + M * K * 2 + M * N * 4 + 32
+
+
+class Clocks:
+    """Samples nvidia-smi during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        self.path = tempfile.mktemp(suffix=".csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def setup_dist():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(v, world):
+    import torch
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# the layer on the GPU
+# ---------------------------------------------------------------------------
+
+def build_layer(dev, cb):
+    import torch
+    import weight_only_bit_gemv_b200 as q4
+    wl = synth.WORKLOADS["llama2_7b_layer"]
+    lins = []
+    for lin in wl.linears:
+        seed = synth.seed_for(wl.index, 0, lin.name)
+        w = synth.weights_device(seed, lin.N, lin.K, wl.w_std, dev)
+        codes, scales = q4.q4_pack(w, cb)
+        del w
+        copies = [(codes, scales)] + [(codes.clone(), scales.clone()) for _ in range(COPIES - 1)]
+        x = synth.activations_device(synth.x_seed(seed), 1, lin.K, dev)
+        y = torch.empty((1, lin.N), dtype=torch.float32, device=dev)
+        lins.append(dict(lin=lin, copies=copies, x=x, y=y, seed=seed))
+    torch.cuda.synchronize()
+    return lins
+
+
+def capture_graphs(lins, cb, stream, with_events):
+    """One CUDA graph per weight copy: the step's four launches, optionally
+    with an event recorded after each launch."""
+    import torch
+    import weight_only_bit_gemv_b200 as q4
+    graphs, events = [], []
+    for c in range(COPIES):
+        g = torch.cuda.CUDAGraph()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(lins) + 1)] if with_events else []
+        with torch.cuda.graph(g, stream=stream):
+            if with_events:
+                evs[0].record()
+            for i, L in enumerate(lins):
+                codes, scales = L["copies"][c]
+                q4.q4_gemv(codes, scales, cb, L["x"], L["y"])
+                if with_events:
+                    evs[i + 1].record()
+        graphs.append(g)
+        events.append(evs)
+    return graphs, events
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import weight_only_bit_gemv_b200 as q4
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    q4.load()
+    hbm_peak, tc_peak, peak_src = peaks()
+    cb = torch.from_numpy(synth.codebook().view(np.int16)).to(dev)
+    lins = build_layer(dev, cb)
+    bytes_step = sum(algo_bytes(1, L["lin"].N, L["lin"].K) for L in lins)
+    stream = torch.cuda.Stream(device=dev)
+
+    # warm-up outside capture (sets kernel attributes), then capture
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            for L in lins:
+                q4.q4_gemv(L["copies"][0][0], L["copies"][0][1], cb, L["x"], L["y"])
+    stream.synchronize()
+    graphs, _ = capture_graphs(lins, cb, stream, with_events=False)
+    egraphs, eevents = capture_graphs(lins, cb, stream, with_events=True)
+
+    K, W = args.steps, args.warmup
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            graphs[i % COPIES].replay()
+    stream.synchronize()
+
+    # ---- timed region: exactly K steps -------------------------------------
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record()
+        for i in range(K):
+            graphs[i % COPIES].replay()
+        t1.record()
+    t1.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms_total = max_over_ranks(t0.elapsed_time(t1), world)
+    ms_step = ms_total / K
+
+    # ---- per-launch durations (graphs with an event after each launch) -------
+    per = [[] for _ in lins]
+    reps = max(COPIES, min(K, 400))
+    with torch.cuda.stream(stream):
+        for i in range(reps):
+            egraphs[i % COPIES].replay()
+            if i % COPIES == COPIES - 1:
+                stream.synchronize()
+                for c in range(COPIES):
+                    evs = eevents[c]
+                    for j in range(len(lins)):
+                        per[j].append(evs[j].elapsed_time(evs[j + 1]))
+    stream.synchronize()
+    per_ms = [statistics.mean(p) for p in per]
+    dom = max(range(len(lins)), key=lambda j: algo_bytes(1, lins[j]["lin"].N, lins[j]["lin"].K))
+    dom_bytes = algo_bytes(1, lins[dom]["lin"].N, lins[dom]["lin"].K)
+    dom_gbs = dom_bytes / (per_ms[dom] * 1e-3) / 1e9
+
+    # ---- end to end through the Python API with host buffers -----------------
+    xh = [torch.empty((1, L["lin"].K), dtype=torch.bfloat16).pin_memory() for L in lins]
+    for h, L in zip(xh, lins):
+        h.copy_(L["x"].cpu())
+    yh = [torch.empty((1, L["lin"].N), dtype=torch.float32).pin_memory() for L in lins]
+    e2e_steps = min(K, 2000)
+    h2d = sum(h.numel() * 2 for h in xh)
+    d2h = sum(h.numel() * 4 for h in yh)
+    with torch.cuda.stream(stream):
+        for i in range(min(W, 20) + 1):
+            for j, L in enumerate(lins):
+                L["x"].copy_(xh[j], non_blocking=True)
+                q4.q4_gemv(L["copies"][0][0], L["copies"][0][1], cb, L["x"], L["y"])
+                yh[j].copy_(L["y"], non_blocking=True)
+    stream.synchronize()
+    barrier(world)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record()
+        for i in range(e2e_steps):
+            c = i % COPIES
+            for j, L in enumerate(lins):
+                L["x"].copy_(xh[j], non_blocking=True)
+                q4.q4_gemv(L["copies"][c][0], L["copies"][c][1], cb, L["x"], L["y"])
+                yh[j].copy_(L["y"], non_blocking=True)
+        e1.record()
+    e1.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+
+    # ---- prefill q4_gemm, M = 256, Llama-2-70B linears --------------------------
+    gemm = None
+    if not args.no_gemm:
+        gemm = bench_prefill(dev, cb, stream, tc_peak, M=256)
+
+    # ---- CPU baseline: the oracle on the host --------------------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(lins, cb, args.cpu_seconds)
+
+    value = world * bytes_step / (ms_step * 1e-3) / 1e9
+    line = {
+        "metric": "q4_gemv HBM GB/s (% of B200 peak) at M=1; q4_gemm TFLOP/s at M>=16",
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(ms_step, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u4 codes x bf16 -> f16 mma, f32 accumulate",
+        "data": "synthetic (seeded N(0,0.02) weights quantized by q4_pack; x ~ N(0,1) bf16)",
+        "config": {
+            "workload": "llama2_7b_layer: qkv 4096->12288, o 4096->4096, gate_up 4096->22016, "
+                        "down 11008->4096; M=1; one q4_gemv per linear",
+            "bytes_per_step": bytes_step,
+            "l2": f"inputs larger than L2: {COPIES} rotating copies of the packed layer "
+                  f"({COPIES * sum(L['copies'][0][0].numel() + 2 * L['copies'][0][1].numel() for L in lins) / 1e6:.0f} MB)",
+            "launch": "CUDA graphs of the step's four launches",
+            "hbm_frac_of_" + peak_src: round(value / world / hbm_peak, 4),
+            "per_linear_us": {L["lin"].name: round(per_ms[j] * 1e3, 3) for j, L in enumerate(lins)},
+            "decode_tok_s_equiv_32_layers": round(1e3 / (ms_step * 32), 1),
+        },
+        "roofline": {
+            "kernel": f"q4_gemv gate_up {lins[dom]['lin'].K}->{lins[dom]['lin'].N}",
+            "bound": "hbm",
+            "achieved": round(dom_gbs, 2),
+            "peak": hbm_peak,
+            "peak_source": peak_src,
+            "unit": "GB/s",
+            "frac": round(dom_gbs / hbm_peak, 4),
+            "traffic": None,
+        },
+        "e2e": {
+            "value": round(world * bytes_step / (e2e_ms * 1e-3) / 1e9, 2),
+            "unit": "GB/s",
+            "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(e2e_ms, 6),
+            "api": "weight_only_bit_gemv_b200.q4_gemv per linear, eager, host x in / host y out",
+        },
+        "gpu_launches": 4 * K,
+        "clocks": clk,
+    }
+    if gemm is not None:
+        line["gemm_prefill"] = gemm
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def bench_prefill(dev, cb, stream, tc_peak, M=256):
+    import torch
+    import weight_only_bit_gemv_b200 as q4
+    wl = synth.WORKLOADS["llama2_70b_prefill"]
+    out = {}
+    total_flop, total_ms = 0.0, 0.0
+    for lin in wl.linears:
+        seed = synth.seed_for(wl.index, 0, lin.name)
+        w = synth.weights_device(seed, lin.N, lin.K, wl.w_std, dev)
+        codes, scales = q4.q4_pack(w, cb)
+        del w
+        x = synth.activations_device(synth.x_seed(seed) + M, M, lin.K, dev)
+        y = torch.empty((M, lin.N), dtype=torch.float32, device=dev)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                q4.q4_gemm(codes, scales, cb, x, y)
+            stream.synchronize()
+            reps = 10
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                q4.q4_gemm(codes, scales, cb, x, y)
+            e1.record()
+        e1.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        flop = 2.0 * M * lin.N * lin.K
+        out[lin.name] = {"us": round(ms * 1e3, 2), "tflops": round(flop / (ms * 1e-3) / 1e12, 2)}
+        total_flop += flop
+        total_ms += ms
+        del codes, scales, x, y
+        torch.cuda.empty_cache()
+    tf = total_flop / (total_ms * 1e-3) / 1e12
+    return {"workload": "llama2_70b_prefill layer (4 linears), M=256", "tflops": round(tf, 2),
+            "frac_of_bf16_peak": round(tf / tc_peak, 4), "per_linear": out,
+            "note": "no L2 flush: each linear is 37-253 MB of packed weights, read once per launch"}
+
+
+def cpu_baseline(lins, cb, seconds):
+    """The oracle, as it stands, single-threaded, on a bounded sample: the first
+    rows of each linear of the same layer (same weights, copied to the host)."""
+    import oracle
+    cbn = synth.codebook()
+    # estimate: the oracle's matmul at M=1 costs ~30 ns/weight on these hosts
+    total_w = sum(L["lin"].N * L["lin"].K for L in lins)
+    frac = min(1.0, seconds / (total_w * 30e-9))
+    packs = []
+    for L in lins:
+        n = max(16, int(L["lin"].N * frac))
+        seed = L["seed"]
+        import torch
+        w = synth.weights_device(seed, L["lin"].N, L["lin"].K, 0.02, L["x"].device)[:n].cpu().numpy()
+        codes, scales = oracle.pack(w, cbn)
+        x = L["x"].cpu().view(torch.int16).numpy().view(np.uint16)
+        packs.append((codes, scales, x, n, L["lin"].K))
+    t = time.perf_counter()
+    byt = 0
+    for codes, scales, x, n, K in packs:
+        oracle.matmul(codes, scales, cbn, x, with_abs=False)
+        byt += algo_bytes(1, n, K)
+    dt = time.perf_counter() - t
+    return {"value": round(byt / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {frac:.1%} of the rows of each of the 4 linears (same seeded "
+                      f"weights, packed by the oracle), M=1, one pass; {dt:.1f} s single-threaded",
+            "host_cpus": os.cpu_count()}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the oracle, single-threaded, on the host cores."""
+    if rank != 0:
+        return
+    import oracle
+    cbn = synth.codebook()
+    wl = synth.WORKLOADS["llama2_7b_layer"]
+    steps = args.steps + args.warmup
+    budget = args.ref_seconds
+    total_w = sum(l.N * l.K for l in wl.linears)
+    frac = min(1.0, budget / steps / (total_w * 30e-9))
+    packs = []
+    for lin in wl.linears:
+        n = max(8, int(lin.N * frac))
+        seed = synth.seed_for(wl.index, 0, lin.name)
+        rng = np.random.Generator(np.random.PCG64(seed))
+        w = (rng.standard_normal((n, lin.K), dtype=np.float32) * np.float32(wl.w_std))
+        codes, scales = oracle.pack(w, cbn)
+        x = synth.activations(synth.x_seed(seed), 1, lin.K)
+        packs.append((codes, scales, x, n, lin.K))
+    byt = sum(algo_bytes(1, n, K) for _, _, _, n, K in packs)
+
+    def step():
+        for codes, scales, x, n, K in packs:
+            oracle.matmul(codes, scales, cbn, x, with_abs=False)
+
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t) / args.steps
+    v = byt / dt / 1e9
+    sample = (f"first {frac:.2%} of the rows of each Llama-2-7B linear per step "
+              f"({byt / 1e6:.2f} MB algorithmic), M=1, single-threaded C oracle")
+    print(json.dumps({
+        "impl": "reference",
+        "metric": "q4_gemv HBM GB/s (% of B200 peak) at M=1; q4_gemm TFLOP/s at M>=16",
+        "value": round(v, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+        "config": {"workload": "llama2_7b_layer: qkv 4096->12288, o 4096->4096, gate_up "
+                               "4096->22016, down 11008->4096; M=1 (row sample)"},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-gemm", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=90.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = setup_dist()
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

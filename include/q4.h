@@ -1,0 +1,152 @@
+/*
+ * q4.h -- C ABI of the weight-only 4-bit codebook linear layer for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operation.  A linear layer y = x * W^T whose weight matrix W [N][K]
+ * (N outputs, K inputs) is stored as 4-bit codes into a 16-entry binary16
+ * codebook, with one binary16 scale per group of 64 consecutive k of a row:
+ *
+ *     W[n][k] = codebook[code(n, k)] * scale[n][k / 64]
+ *
+ * This is the layout the "deep-fold" page describes in its "Method" section
+ * (each group of 64 weights stores four-bit NF4 codes and one FP16 scale;
+ * the packed payload is about 3.76x smaller than BF16).  The matmul entry
+ * points rebuild W inside the kernel while they multiply, reading the codes
+ * "straight out of the codebook" ("Trapetum" overview, "What it does"), and
+ * never write a dense W to memory ("Trapetum" landing page, opening
+ * paragraph; "deep-fold", "Method").  Decode (one token) is a GEMV and
+ * prompt processing a tensor-core GEMM ("deep-fold", "Method" table).
+ *
+ * Layouts (all row-major and contiguous; there are no stride arguments):
+ *   codes    uint8_t  [N][K/2]   byte j of row n holds code(n, 2j) in its low
+ *                                nibble and code(n, 2j+1) in its high nibble
+ *   scales   uint16_t [N][K/64]  binary16 bit patterns
+ *   codebook uint16_t [16]       binary16 bit patterns (any values, any order)
+ *   x        uint16_t [M][K]     bfloat16 bit patterns (M tokens)
+ *   y        float    [M][N]     binary32, fully overwritten
+ *   w        float    [N][K]     binary32 (input of q4_pack, output of q4_dequant)
+ *
+ * Ownership.  Every pointer is device memory owned by the caller (PyTorch,
+ * cudaMalloc, ...).  The library allocates nothing, keeps no pointer after a
+ * call returns, and holds only a per-device cache of the device's properties.
+ * All calls are asynchronous on the caller's stream (0 = legacy default
+ * stream); none synchronizes the host.  Inputs and outputs must not overlap.
+ * The calls are thread-safe.
+ *
+ * Errors.  Each call validates its arguments before launching anything, in
+ * this order, and returns the first failure:
+ *   Q4_ERR_SHAPE  K <= 0, K not a multiple of 64, K > Q4_MAX_K, M < 0, N < 0,
+ *                 M or N above Q4_MAX_MN, or (q4_gemv only) M != 1
+ *   (M == 0 or N == 0 is valid: Q4_OK is returned and nothing is launched)
+ *   Q4_ERR_NULL   a required pointer is NULL
+ *   Q4_ERR_ALIGN  a pointer is not 16-byte aligned
+ *   Q4_ERR_ARCH   the current device is not compute capability 10.0 (sm_100)
+ *   Q4_ERR_CUDA   a CUDA runtime call or the kernel launch failed; the CUDA
+ *                 error code is available from q4_last_cuda_error()
+ * Faults that happen while a kernel runs surface, as with any CUDA kernel, at
+ * the caller's next synchronization.
+ *
+ * Input domain.  w finite with |w| <= 65504; x finite with |x| <= 65504; a
+ * finite codebook.  Outside it results are unspecified.
+ */
+#ifndef Q4_H
+#define Q4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t (a CUstream_st pointer); pass a cudaStream_t. */
+typedef struct CUstream_st* q4_stream_t;
+
+typedef enum {
+    Q4_OK = 0,
+    Q4_ERR_NULL = 1,
+    Q4_ERR_SHAPE = 2,
+    Q4_ERR_ALIGN = 3,
+    Q4_ERR_ARCH = 4,
+    Q4_ERR_CUDA = 5
+} q4_status;
+
+#define Q4_ABI_VERSION 1
+#define Q4_GROUP 64
+#define Q4_MAX_K (1 << 20)
+#define Q4_MAX_MN 2147483647LL
+
+/*
+ * q4_pack -- quantize a dense binary32 W [N][K] into codes and scales.
+ * Source: "deep-fold", "Method" (64-weight groups, four-bit codes, one FP16
+ * scale; a CPU compressor writes them).  Per group of 64:
+ *   scale = binary16(max |w|), rounded to nearest-even;
+ *   code  = argmin_i |w / scale - codebook[i]|, the division and distances in
+ *           binary32 (IEEE, round to nearest-even), ties to the lowest i;
+ *   a scale that rounds to 0 gives every weight the index of the codebook
+ *   entry of smallest magnitude.
+ * Results are bit-identical to a serial IEEE implementation of these steps.
+ * In: w [N][K] fp32, codebook [16].  Out: codes [N][K/2], scales [N][K/64].
+ */
+q4_status q4_pack(const float* w, const uint16_t* codebook, uint8_t* codes,
+                  uint16_t* scales, int64_t N, int64_t K, q4_stream_t stream);
+
+/*
+ * q4_dequant -- write the dense binary32 W [N][K] = codebook[code] * scale.
+ * The product of two binary16 values is exact in binary32, so the output is
+ * exact.  For checking and debugging: the matmul entry points never call it.
+ * In: codes, scales, codebook.  Out: w_out [N][K] fp32.
+ */
+q4_status q4_dequant(const uint8_t* codes, const uint16_t* scales,
+                     const uint16_t* codebook, float* w_out, int64_t N,
+                     int64_t K, q4_stream_t stream);
+
+/*
+ * q4_gemv -- one-token decode: y[0][n] = sum_k W[n][k] * x[0][k], M must be 1.
+ * Source: "deep-fold", "Method" table (decode: a CUDA-core NF4 GEMV that
+ * rebuilds values while it multiplies); "Trapetum" overview, "The bandwidth
+ * law" (decode speed is set by the bytes of weights read).
+ * Each weight is rebuilt in registers as binary16 codebook[code]; products
+ * with x are exact and accumulate in binary32; the group's scale multiplies
+ * the group's binary32 partial sum.  The result matches the exact sum to
+ * within 1e-4 * sum_k |W x| + 1e-6 per element.
+ * In: codes, scales, codebook, x [1][K] bf16.  Out: y [1][N] fp32.
+ */
+q4_status q4_gemv(const uint8_t* codes, const uint16_t* scales,
+                  const uint16_t* codebook, const uint16_t* x, float* y,
+                  int64_t M, int64_t N, int64_t K, q4_stream_t stream);
+
+/*
+ * q4_gemm -- M tokens at once: y[m][n] = sum_k W[n][k] * x[m][k], any M >= 0.
+ * Source: "deep-fold", "Method" table (prompt processing: a tensor-core NF4
+ * GEMM that rebuilds weights into fragments); "Trapetum" overview, "What it
+ * does" (speculative decoding verifies a few drafted tokens at once).
+ * M <= 16 (verify batches) runs the same kernel family as q4_gemv, exact
+ * products with binary32 accumulation.  M > 16 (prefill chunks) runs a tcgen05
+ * tensor-core kernel: each weight is rebuilt as binary16(codebook * scale),
+ * x is rounded to binary16, and products accumulate in binary32 in tensor
+ * memory.  Either way the result is within 1e-4 * sum_k |W x| + 1e-6 of the
+ * exact sum per element (for the tensor-core path this holds statistically:
+ * the binary16 rounding of W and x is a relative error of at most 2^-11 per
+ * term, far inside the bound once K is a few hundred).
+ * In: codes, scales, codebook, x [M][K] bf16.  Out: y [M][N] fp32.
+ */
+q4_status q4_gemm(const uint8_t* codes, const uint16_t* scales,
+                  const uint16_t* codebook, const uint16_t* x, float* y,
+                  int64_t M, int64_t N, int64_t K, q4_stream_t stream);
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* q4_status_string(q4_status status);
+
+/* The cudaError_t value behind the last Q4_ERR_CUDA returned on this thread
+ * (0 if none). */
+int q4_last_cuda_error(void);
+
+/* Q4_ABI_VERSION of the library that was loaded. */
+int q4_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* Q4_H */

@@ -130,6 +130,26 @@ def codebook() -> np.ndarray:
     return np.array(vals, dtype=np.uint16)
 
 
+def weights_device(seed: int, N: int, K: int, std: float, device):
+    """W [N, K] float32 ~ N(0, std^2) drawn on a CUDA device with torch's seeded
+    generator (Philox); used where host generation of hundreds of millions of
+    samples would dominate the run time.  Same distribution as ``weights``,
+    different stream."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    w = torch.randn((N, K), generator=g, device=device, dtype=torch.float32)
+    return w.mul_(std)
+
+
+def activations_device(seed: int, M: int, K: int, device):
+    """x [M, K] bfloat16 ~ N(0, 1) drawn on a CUDA device (rounded to nearest-even)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return torch.randn((M, K), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+
 def integer_codebook() -> np.ndarray:
     """Codebook {-8, ..., 7} (exact in binary16), used for exact-arithmetic checks."""
     return f32_to_f16_bits(np.arange(-8, 8, dtype=np.float32))

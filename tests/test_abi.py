@@ -1,0 +1,88 @@
+"""The C-ABI library: it loads, exports every function include/q4.h declares,
+and rejects bad arguments on the host before touching CUDA.
+
+These run without a GPU: every call below returns from argument validation,
+which happens before any CUDA runtime call (q4.h, "Errors")."""
+import ctypes
+import subprocess
+
+import pytest
+
+import weight_only_bit_gemv_b200 as q4
+
+OK, NULL, SHAPE, ALIGN = 0, 1, 2, 3
+A = 1 << 20          # a 16-byte-aligned fake address; never dereferenced
+MIS = A + 8          # misaligned
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return q4.load()
+
+
+def test_exports_every_declared_function(lib):
+    names = q4.header_functions()
+    assert {"q4_pack", "q4_dequant", "q4_gemv", "q4_gemm", "q4_status_string",
+            "q4_last_cuda_error", "q4_abi_version"} <= set(names)
+    out = subprocess.run(["nm", "-D", "--defined-only", q4.library_path()],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(lib, n)
+
+
+def test_abi_version_and_strings(lib):
+    assert q4.abi_version() == 1
+    for code in range(6):
+        s = q4.status_string(code)
+        assert s.startswith(q4.STATUS[code])
+    assert "unknown" in q4.status_string(99)
+    assert lib.q4_last_cuda_error() == 0
+
+
+def test_gemv_rejects_shapes(lib):
+    f = lib.q4_gemv
+    assert f(A, A, A, A, A, 2, 64, 256, None) == SHAPE        # M != 1
+    assert f(A, A, A, A, A, 1, 64, 100, None) == SHAPE        # K % 64
+    assert f(A, A, A, A, A, 1, 64, 0, None) == SHAPE          # K == 0
+    assert f(A, A, A, A, A, 1, -1, 64, None) == SHAPE         # N < 0
+    assert f(A, A, A, A, A, 1, 64, (1 << 20) + 64, None) == SHAPE   # K > Q4_MAX_K
+    assert f(A, A, A, A, A, 1, 0, 64, None) == OK             # empty: no launch
+    assert f(None, None, None, None, None, 1, 0, 64, None) == OK
+
+
+def test_gemm_rejects(lib):
+    f = lib.q4_gemm
+    assert f(A, A, A, A, A, -1, 64, 64, None) == SHAPE
+    assert f(A, A, A, A, A, 0, 64, 64, None) == OK
+    assert f(A, A, A, A, A, 5, 0, 64, None) == OK
+    assert f(None, A, A, A, A, 5, 64, 64, None) == NULL
+    assert f(A, A, A, A, None, 5, 64, 64, None) == NULL
+    assert f(A, MIS, A, A, A, 5, 64, 64, None) == ALIGN
+    assert f(A, A, A, MIS, A, 5, 64, 64, None) == ALIGN
+    assert f(A, A, A, A, MIS, 5, 64, 64, None) == ALIGN
+    assert f(A, A, MIS, A, A, 5, 64, 64, None) == ALIGN
+
+
+def test_pack_dequant_reject(lib):
+    assert lib.q4_pack(A, A, A, A, 4, 96, None) == SHAPE
+    assert lib.q4_pack(A, A, A, A, -4, 64, None) == SHAPE
+    assert lib.q4_pack(A, A, A, A, 0, 64, None) == OK
+    assert lib.q4_pack(A, None, A, A, 4, 64, None) == NULL
+    assert lib.q4_pack(A, A, MIS, A, 4, 64, None) == ALIGN
+    assert lib.q4_dequant(A, A, A, A, 4, 32, None) == SHAPE
+    assert lib.q4_dequant(A, A, A, None, 4, 64, None) == NULL
+    assert lib.q4_dequant(MIS, A, A, A, 4, 64, None) == ALIGN
+    assert lib.q4_dequant(A, A, A, A, 0, 64, None) == OK
+
+
+def test_binding_marshalling_checks():
+    import torch
+    cpu = torch.zeros(4, 32, dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        q4.q4_gemv(cpu, torch.zeros(4, 1, dtype=torch.float16), torch.zeros(16, dtype=torch.float16),
+                   torch.zeros(1, 64, dtype=torch.bfloat16))
+    with pytest.raises(TypeError):
+        q4.q4_pack(torch.zeros(4, 64, dtype=torch.float64), torch.zeros(16, dtype=torch.float16))

@@ -1,0 +1,275 @@
+"""GPU parity: the CUDA kernels, called through the C ABI, against the oracle.
+
+Bars: q4_pack and q4_dequant bit-exact; q4_gemv / q4_gemm within
+|y - y_ref| <= 1e-4 * sum_k |W x| + 1e-6 per element; exact-arithmetic cases
+(integer codebook, power-of-two scales, small-integer x; one-hot x; zero
+scales) bit-exact on every path.  Inputs come from ``synth`` (seeded) or are
+built here; expected values come only from the oracle.
+"""
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import weight_only_bit_gemv_b200 as q4
+from helpers import GROUP, pack_codes, within_tolerance
+
+pytestmark = pytest.mark.gpu
+
+NF4 = synth.codebook()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+    q4.load()
+
+
+def dev_u16(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+def dev_u8(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host_u16(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint16)
+
+
+def run_matmul(codes, scales, cb, x, path="gemm"):
+    """codes/scales/cb/x numpy -> y numpy via q4_gemv (M = 1) or q4_gemm."""
+    M, N = x.shape[0], codes.shape[0]
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    fn = q4.q4_gemv if path == "gemv" else q4.q4_gemm
+    fn(dev_u8(codes), dev_u16(scales), dev_u16(cb), dev_u16(x), y)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+def assert_close(y, codes, scales, cb, x, rows=None, label=""):
+    y_ref, a = oracle.matmul(codes, scales, cb, x, rows=rows)
+    ys = y if rows is None else y[:, rows]
+    ok, worst = within_tolerance(ys, y_ref, a)
+    assert ok, f"{label}: worst err/bound = {worst:.3g}"
+    return worst
+
+
+def random_packed(seed, N, K, pow2_scales=False):
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    if pow2_scales:
+        scales = np.asarray(2.0 ** rng.integers(-6, 2, size=(N, K // GROUP)), np.float16).view(np.uint16)
+    else:
+        scales = synth.f32_to_f16_bits(rng.uniform(0.005, 0.05, size=(N, K // GROUP)).astype(np.float32))
+    return codes, scales
+
+
+# ---------------------------------------------------------------------------
+# pack / dequant: bit-exact
+# ---------------------------------------------------------------------------
+
+def gpu_pack(w, cb):
+    codes, scales = q4.q4_pack(torch.from_numpy(w).cuda(), dev_u16(cb))
+    torch.cuda.synchronize()
+    return codes.cpu().numpy(), scales.cpu().numpy().view(np.uint16)
+
+
+def gpu_dequant(codes, scales, cb):
+    w = q4.q4_dequant(dev_u8(codes), dev_u16(scales), dev_u16(cb))
+    torch.cuda.synchronize()
+    return w.cpu().numpy()
+
+
+@pytest.mark.parametrize("N,K", [(128, 256), (1, 64), (37, 448), (300, 4096)])
+def test_pack_dequant_bit_exact(N, K):
+    w = synth.weights(7 + N, N, K, 0.02)
+    c_ref, s_ref = oracle.pack(w, NF4)
+    c, s = gpu_pack(w, NF4)
+    assert np.array_equal(s, s_ref) and np.array_equal(c, c_ref)
+    wd = gpu_dequant(c_ref, s_ref, NF4)
+    assert np.array_equal(wd.view(np.uint32), oracle.dequant(c_ref, s_ref, NF4).view(np.uint32))
+
+
+def test_pack_edge_cases():
+    K = 8 * GROUP
+    rng = np.random.default_rng(1)
+    w = (rng.standard_normal((6, K)) * 0.02).astype(np.float32)
+    w[0] = 0.0                                    # zero groups
+    w[1, :GROUP] = 1e-9                           # scale underflows to 0
+    w[1, GROUP:2 * GROUP] *= 1e-4                 # subnormal binary16 scales
+    w[2] = rng.uniform(-65504, 65504, size=K)     # extreme magnitudes
+    w[2, 0] = 65504.0
+    w[3] = np.linspace(-1, 1, K)                  # dense sweep across codes
+    w[4, :GROUP] = 8.0 * np.array([1, 0.5, -0.5] + [0.1875] * (GROUP - 3), np.float32)
+    w[5] = -0.0
+    for cb in (NF4, synth.integer_codebook(), NF4[rng.permutation(16)]):
+        c_ref, s_ref = oracle.pack(w, cb)
+        c, s = gpu_pack(w, cb)
+        assert np.array_equal(s, s_ref) and np.array_equal(c, c_ref)
+        wd = gpu_dequant(c_ref, s_ref, cb)
+        assert np.array_equal(wd.view(np.uint32), oracle.dequant(c_ref, s_ref, cb).view(np.uint32))
+
+
+def test_pack_round_trip_on_gpu():
+    """Weights on cb * s with an end code per group re-pack to the same codes."""
+    rng = np.random.default_rng(2)
+    N, K = 64, 1024
+    c = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    c[:, ::GROUP] = 15
+    s = rng.uniform(0.001, 2.0, size=(N, K // GROUP)).astype(np.float16)
+    cbv = NF4.view(np.float16).astype(np.float64)
+    w = (cbv[c] * np.repeat(s.astype(np.float64), GROUP, axis=1)).astype(np.float32)
+    codes, scales = gpu_pack(w, NF4)
+    assert np.array_equal(scales, s.view(np.uint16)) and np.array_equal(codes, pack_codes(c))
+
+
+# ---------------------------------------------------------------------------
+# matmul: exact special cases on every path
+# ---------------------------------------------------------------------------
+
+ALL_M = [1, 2, 3, 8, 9, 16, 17, 32, 40, 128]
+
+
+@pytest.mark.parametrize("M", ALL_M)
+def test_integer_codebook_exact(M):
+    rng = np.random.default_rng(100 + M)
+    N, K = 200, 1024
+    cb = synth.integer_codebook()
+    codes = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    scales = np.asarray(2.0 ** rng.integers(0, 3, size=(N, K // GROUP)), np.float16).view(np.uint16)
+    x = synth.f32_to_bf16_bits(rng.integers(-4, 5, size=(M, K)).astype(np.float32))
+    y_ref, _ = oracle.matmul(codes, scales, cb, x)
+    y = run_matmul(codes, scales, cb, x)
+    assert np.array_equal(y, y_ref)
+    if M == 1:
+        assert np.array_equal(run_matmul(codes, scales, cb, x, "gemv"), y_ref)
+
+
+@pytest.mark.parametrize("M", [1, 5, 16, 33])
+def test_one_hot_selects_column(M):
+    N, K = 96, 512
+    codes, scales = random_packed(5, N, K, pow2_scales=True)
+    W = oracle.dequant(codes, scales, NF4)
+    ks = (np.arange(M) * 37) % K
+    x = np.zeros((M, K), np.uint16)
+    x[np.arange(M), ks] = 0x3F80
+    y = run_matmul(codes, scales, NF4, x)
+    assert np.array_equal(y, W[:, ks].T)
+
+
+@pytest.mark.parametrize("M", [1, 4, 24])
+def test_zero_scales_give_zero(M):
+    N, K = 50, 256
+    codes, _ = random_packed(6, N, K)
+    scales = np.zeros((N, K // GROUP), np.uint16)
+    x = synth.activations(9, M, K)
+    assert np.all(run_matmul(codes, scales, NF4, x) == 0.0)
+
+
+# ---------------------------------------------------------------------------
+# matmul: tolerance, ragged and edge shapes
+# ---------------------------------------------------------------------------
+
+def test_tiny_config_gemv():
+    """One 4-bit layer, K=256, N=128, M=1; uniform codes, scales U[0.005, 0.05]."""
+    wl = synth.WORKLOADS["tiny"]
+    lin = wl.linears[0]
+    seed = synth.seed_for(wl.index, 0, lin.name)
+    codes, scales = synth.tiny_codes_scales(seed, lin.N, lin.K)
+    x = synth.activations(synth.x_seed(seed), 1, lin.K)
+    assert_close(run_matmul(codes, scales, NF4, x, "gemv"), codes, scales, NF4, x, label="tiny")
+
+
+@pytest.mark.parametrize("M,N,K", [
+    (1, 1, 64), (1, 7, 128), (1, 17, 448), (1, 1000, 4160), (1, 33, 28672),
+    (3, 100, 192), (8, 129, 1024), (9, 31, 2048), (16, 300, 4096), (16, 64, 14336),
+    (17, 130, 512), (64, 257, 1088), (100, 96, 4096)])
+def test_ragged_shapes(M, N, K):
+    codes, scales = random_packed(M * 1000 + N, N, K)
+    x = synth.activations(K + N, M, K)
+    y = run_matmul(codes, scales, NF4, x, "gemv" if M == 1 else "gemm")
+    assert_close(y, codes, scales, NF4, x, label=f"M{M} N{N} K{K}")
+
+
+def test_output_bounds_and_stream():
+    """Writes stay inside y; a side stream is honoured."""
+    M, N, K = 3, 77, 640
+    codes, scales = random_packed(11, N, K)
+    x = synth.activations(12, M, K)
+    buf = torch.full((M * N + 64,), 12345.0, dtype=torch.float32, device="cuda")
+    y = buf[:M * N].view(M, N)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        q4.q4_gemm(dev_u8(codes), dev_u16(scales), dev_u16(NF4), dev_u16(x), y)
+    s.synchronize()
+    assert torch.all(buf[M * N:] == 12345.0)
+    assert_close(y.cpu().numpy(), codes, scales, NF4, x, label="stream")
+
+
+# ---------------------------------------------------------------------------
+# the workloads at full size
+# ---------------------------------------------------------------------------
+
+@functools.lru_cache(maxsize=None)
+def packed_linear(workload: str, linear: str, layer: int = 0):
+    """Seeded W of one linear, quantized by the oracle; W is kept only where the
+    GPU pack is compared against it."""
+    wl = synth.WORKLOADS[workload]
+    lin = {l.name: l for l in wl.linears}[linear]
+    seed = synth.seed_for(wl.index, layer, lin.name)
+    w = synth.weights(seed, lin.N, lin.K, wl.w_std)
+    codes, scales = oracle.pack(w, NF4)
+    keep = workload != "llama2_70b_prefill" and linear != "lm_head"
+    return (w if keep else w[:1].copy()), codes, scales, seed
+
+
+@pytest.mark.parametrize("linear", ["qkv", "o", "gate_up", "down"])
+def test_llama2_7b_layer_full(linear):
+    """Every output of each Llama-2-7B linear at M = 1; pack compared in full."""
+    w, codes, scales, seed = packed_linear("llama2_7b_layer", linear)
+    c, s = gpu_pack(w, NF4)
+    assert np.array_equal(s, scales) and np.array_equal(c, codes)
+    x = synth.activations(synth.x_seed(seed), 1, w.shape[1])
+    assert_close(run_matmul(codes, scales, NF4, x, "gemv"), codes, scales, NF4, x, label=linear)
+
+
+@pytest.mark.parametrize("linear", ["qkv", "o", "gate_up", "down", "lm_head"])
+def test_llama31_8b_step_shapes_full(linear):
+    """Layer 0 of the Llama-3.1-8B step and the lm_head, every output at M = 1."""
+    w, codes, scales, seed = packed_linear("llama31_8b_step", linear)
+    if linear != "lm_head":
+        c, s = gpu_pack(w, NF4)
+        assert np.array_equal(s, scales) and np.array_equal(c, codes)
+    x = synth.activations(synth.x_seed(seed), 1, codes.shape[1] * 2)
+    assert_close(run_matmul(codes, scales, NF4, x, "gemv"), codes, scales, NF4, x, label=linear)
+
+
+@pytest.mark.parametrize("M", [2, 4, 8, 16])
+@pytest.mark.parametrize("linear", ["qkv", "o", "gate_up", "down", "lm_head"])
+def test_small_m_verify(linear, M):
+    """Verify batches on the Llama-3.1-8B shapes: all M rows x 2048 sampled outputs."""
+    w, codes, scales, seed = packed_linear("llama31_8b_step", linear)
+    x = synth.activations(synth.x_seed(seed) + M, M, codes.shape[1] * 2)
+    y = run_matmul(codes, scales, NF4, x)
+    rows = np.random.default_rng(M).choice(codes.shape[0], size=2048, replace=False)
+    assert_close(y, codes, scales, NF4, x, rows=rows, label=f"{linear} M={M}")
+
+
+@pytest.mark.parametrize("M", [32, 128, 256, 512])
+@pytest.mark.parametrize("linear", ["qkv", "o", "gate_up", "down"])
+def test_llama2_70b_prefill(linear, M):
+    """Prefill chunks on Llama-2-70B shapes: all M rows x 256 sampled outputs."""
+    w, codes, scales, seed = packed_linear("llama2_70b_prefill", linear)
+    x = synth.activations(synth.x_seed(seed) + M, M, codes.shape[1] * 2)
+    y = run_matmul(codes, scales, NF4, x)
+    assert np.all(np.isfinite(y))
+    rows = np.random.default_rng(M + 1).choice(codes.shape[0], size=256, replace=False)
+    assert_close(y, codes, scales, NF4, x, rows=rows, label=f"{linear} M={M}")

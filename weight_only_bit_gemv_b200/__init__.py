@@ -1,0 +1,188 @@
+"""Python binding of the sm_100a 4-bit codebook linear-layer library (libq4.so).
+
+Argument marshalling only: every step of pack, dequant and the matmuls runs in
+the CUDA kernels of libq4.so, on the tensors' device, on the current torch
+stream.  PyTorch supplies device memory and streams.  There is no CPU path:
+if the library cannot be loaded, every call raises.
+
+Tensor conventions (all contiguous, on one CUDA device):
+  w        float32            [N, K]
+  codebook float16 or uint16  [16]       (binary16 bits)
+  codes    uint8              [N, K/2]   low nibble = even k
+  scales   float16 or uint16  [N, K/64]  (binary16 bits)
+  x        bfloat16 or uint16 [M, K]     (bfloat16 bits)
+  y        float32            [M, N]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+from . import build as _build
+
+GROUP = 64
+_HERE = os.path.dirname(os.path.abspath(__file__))
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "q4.h")
+
+STATUS = {0: "Q4_OK", 1: "Q4_ERR_NULL", 2: "Q4_ERR_SHAPE", 3: "Q4_ERR_ALIGN", 4: "Q4_ERR_ARCH",
+          5: "Q4_ERR_CUDA"}
+
+
+class Q4Error(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIBRARY
+
+
+def load(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libq4.so (building it with nvcc first if it is missing or stale)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if build_if_missing and _build.stale():
+        _build.build()
+    if not os.path.exists(_build.LIBRARY):
+        raise RuntimeError(f"libq4.so not found at {_build.LIBRARY}; run "
+                           "python -m weight_only_bit_gemv_b200.build")
+    lib = ctypes.CDLL(_build.LIBRARY)
+    P, I64, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p
+    lib.q4_pack.argtypes = [P, P, P, P, I64, I64, S]
+    lib.q4_dequant.argtypes = [P, P, P, P, I64, I64, S]
+    lib.q4_gemv.argtypes = [P, P, P, P, P, I64, I64, I64, S]
+    lib.q4_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, S]
+    for f in ("q4_pack", "q4_dequant", "q4_gemv", "q4_gemm"):
+        getattr(lib, f).restype = ctypes.c_int
+    lib.q4_status_string.argtypes = [ctypes.c_int]
+    lib.q4_status_string.restype = ctypes.c_char_p
+    lib.q4_last_cuda_error.argtypes = []
+    lib.q4_last_cuda_error.restype = ctypes.c_int
+    lib.q4_abi_version.argtypes = []
+    lib.q4_abi_version.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def header_functions() -> list:
+    """Names of the functions include/q4.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(q4_[a-z0-9_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    return load().q4_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        lib = load()
+        msg = f"{what}: {status_string(status)}"
+        if status == 5:
+            msg += f" (cudaError {lib.q4_last_cuda_error()})"
+        raise Q4Error(status, msg)
+
+
+def _stream(t: torch.Tensor, stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(t.device)
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need(t: torch.Tensor, name: str, dtypes, shape=None) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype} not in {dtypes}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)} != {tuple(shape)}")
+
+
+_H16 = (torch.float16, torch.uint16, torch.int16)
+_BF16 = (torch.bfloat16, torch.uint16, torch.int16)
+
+
+def _packed_dims(codes: torch.Tensor):
+    if codes.dim() != 2:
+        raise ValueError("codes must be [N, K/2]")
+    return codes.shape[0], codes.shape[1] * 2
+
+
+def q4_pack(w: torch.Tensor, codebook: torch.Tensor, codes: torch.Tensor = None,
+            scales: torch.Tensor = None, stream=None):
+    """Quantize w [N, K] fp32 into (codes, scales); allocates them with torch if not given."""
+    if w.dim() != 2:
+        raise ValueError("w must be [N, K]")
+    N, K = w.shape
+    if codes is None:
+        codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty((N, K // GROUP), dtype=torch.float16, device=w.device)
+    _need(w, "w", (torch.float32,))
+    _need(codebook, "codebook", _H16, (16,))
+    _need(codes, "codes", (torch.uint8,), (N, K // 2))
+    _need(scales, "scales", _H16, (N, K // GROUP))
+    st = load().q4_pack(w.data_ptr(), codebook.data_ptr(), codes.data_ptr(), scales.data_ptr(),
+                        N, K, _stream(w, stream))
+    _check(st, "q4_pack")
+    return codes, scales
+
+
+def q4_dequant(codes: torch.Tensor, scales: torch.Tensor, codebook: torch.Tensor,
+               w_out: torch.Tensor = None, stream=None) -> torch.Tensor:
+    N, K = _packed_dims(codes)
+    if w_out is None:
+        w_out = torch.empty((N, K), dtype=torch.float32, device=codes.device)
+    _need(codes, "codes", (torch.uint8,))
+    _need(scales, "scales", _H16, (N, K // GROUP))
+    _need(codebook, "codebook", _H16, (16,))
+    _need(w_out, "w_out", (torch.float32,), (N, K))
+    st = load().q4_dequant(codes.data_ptr(), scales.data_ptr(), codebook.data_ptr(),
+                           w_out.data_ptr(), N, K, _stream(codes, stream))
+    _check(st, "q4_dequant")
+    return w_out
+
+
+def _matmul(fn: str, codes, scales, codebook, x, y, stream):
+    N, K = _packed_dims(codes)
+    if x.dim() != 2 or x.shape[1] != K:
+        raise ValueError(f"x must be [M, {K}]")
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=codes.device)
+    _need(codes, "codes", (torch.uint8,))
+    _need(scales, "scales", _H16, (N, K // GROUP))
+    _need(codebook, "codebook", _H16, (16,))
+    _need(x, "x", _BF16)
+    _need(y, "y", (torch.float32,), (M, N))
+    st = getattr(load(), fn)(codes.data_ptr(), scales.data_ptr(), codebook.data_ptr(),
+                             x.data_ptr(), y.data_ptr(), M, N, K, _stream(codes, stream))
+    _check(st, fn)
+    return y
+
+
+def q4_gemv(codes, scales, codebook, x, y=None, stream=None) -> torch.Tensor:
+    """y [1, N] = x [1, K] @ W^T with W rebuilt from codes/scales/codebook in the kernel."""
+    return _matmul("q4_gemv", codes, scales, codebook, x, y, stream)
+
+
+def q4_gemm(codes, scales, codebook, x, y=None, stream=None) -> torch.Tensor:
+    """y [M, N] = x [M, K] @ W^T for any M (M <= 16: verify batches; M > 16: prefill)."""
+    return _matmul("q4_gemm", codes, scales, codebook, x, y, stream)
+
+
+def abi_version() -> int:
+    return load().q4_abi_version()

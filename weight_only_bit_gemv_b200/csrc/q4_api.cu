@@ -1,0 +1,191 @@
+// q4_api.cu -- the C ABI of q4.h: argument validation, the architecture
+// gate, a per-device property cache, and dispatch to the kernel launchers.
+#include <atomic>
+#include <mutex>
+
+#include "q4_internal.cuh"
+
+namespace q4 {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxSlots = 64;
+
+struct Cache {
+    std::mutex mu;
+    bool valid[kMaxDevices] = {};
+    DeviceInfo info[kMaxDevices];
+    std::atomic<int> smem_done[kMaxDevices][kMaxSlots];
+    Cache() {
+        for (auto& row : smem_done)
+            for (auto& v : row) v.store(0, std::memory_order_relaxed);
+    }
+};
+
+Cache& cache() {
+    static Cache c;
+    return c;
+}
+
+thread_local int g_last_cuda_error = 0;
+
+q4_status cuda_fail(cudaError_t e) {
+    g_last_cuda_error = static_cast<int>(e);
+    return Q4_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+q4_status check_K(int64_t K) {
+    if (K <= 0 || K % kGroup != 0 || K > Q4_MAX_K) return Q4_ERR_SHAPE;
+    return Q4_OK;
+}
+
+// Architecture gate plus property lookup for the current device.
+q4_status gate(DeviceInfo* dev) {
+    cudaError_t e = current_device_info(dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev->cc_major != 10 || dev->cc_minor != 0) return Q4_ERR_ARCH;
+    return Q4_OK;
+}
+
+q4_status after_launch(cudaError_t e) {
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+    return Q4_OK;
+}
+
+q4_status check_matmul(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                       const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
+                       bool* empty) {
+    *empty = false;
+    q4_status st = check_K(K);
+    if (st != Q4_OK) return st;
+    if (M < 0 || N < 0 || M > Q4_MAX_MN || N > Q4_MAX_MN) return Q4_ERR_SHAPE;
+    if (M == 0 || N == 0) {
+        *empty = true;
+        return Q4_OK;
+    }
+    if (!codes || !scales || !cb || !x || !y) return Q4_ERR_NULL;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(cb) || !aligned16(x) ||
+        !aligned16(y))
+        return Q4_ERR_ALIGN;
+    return Q4_OK;
+}
+
+}  // namespace
+
+cudaError_t current_device_info(DeviceInfo* info) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    Cache& c = cache();
+    std::lock_guard<std::mutex> lock(c.mu);
+    if (!c.valid[dev]) {
+        DeviceInfo d{};
+        d.device = dev;
+        if ((e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev)) ||
+            (e = cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) ||
+            (e = cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) ||
+            (e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                        dev)))
+            return e;
+        c.info[dev] = d;
+        c.valid[dev] = true;
+    }
+    *info = c.info[dev];
+    return cudaSuccess;
+}
+
+cudaError_t ensure_smem_attr(const void* func, int bytes, int slot, int device) {
+    if (slot < 0 || slot >= kMaxSlots || device < 0 || device >= kMaxDevices)
+        return cudaErrorInvalidValue;
+    std::atomic<int>& done = cache().smem_done[device][slot];
+    if (done.load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) {
+        int prev = done.load(std::memory_order_relaxed);
+        while (prev < bytes && !done.compare_exchange_weak(prev, bytes)) {
+        }
+    }
+    return e;
+}
+
+}  // namespace q4
+
+using namespace q4;
+
+extern "C" {
+
+q4_status q4_pack(const float* w, const uint16_t* codebook, uint8_t* codes, uint16_t* scales,
+                  int64_t N, int64_t K, q4_stream_t stream) {
+    q4_status st = check_K(K);
+    if (st != Q4_OK) return st;
+    if (N < 0 || N > Q4_MAX_MN) return Q4_ERR_SHAPE;
+    if (N == 0) return Q4_OK;
+    if (!w || !codebook || !codes || !scales) return Q4_ERR_NULL;
+    if (!aligned16(w) || !aligned16(codebook) || !aligned16(codes) || !aligned16(scales))
+        return Q4_ERR_ALIGN;
+    DeviceInfo dev;
+    if ((st = gate(&dev)) != Q4_OK) return st;
+    return after_launch(launch_pack(w, codebook, codes, scales, N, K, stream, dev));
+}
+
+q4_status q4_dequant(const uint8_t* codes, const uint16_t* scales, const uint16_t* codebook,
+                     float* w_out, int64_t N, int64_t K, q4_stream_t stream) {
+    q4_status st = check_K(K);
+    if (st != Q4_OK) return st;
+    if (N < 0 || N > Q4_MAX_MN) return Q4_ERR_SHAPE;
+    if (N == 0) return Q4_OK;
+    if (!codes || !scales || !codebook || !w_out) return Q4_ERR_NULL;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(codebook) || !aligned16(w_out))
+        return Q4_ERR_ALIGN;
+    DeviceInfo dev;
+    if ((st = gate(&dev)) != Q4_OK) return st;
+    return after_launch(launch_dequant(codes, scales, codebook, w_out, N, K, stream, dev));
+}
+
+q4_status q4_gemv(const uint8_t* codes, const uint16_t* scales, const uint16_t* codebook,
+                  const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
+                  q4_stream_t stream) {
+    if (M != 1) return Q4_ERR_SHAPE;
+    bool empty;
+    q4_status st = check_matmul(codes, scales, codebook, x, y, M, N, K, &empty);
+    if (st != Q4_OK || empty) return st;
+    DeviceInfo dev;
+    if ((st = gate(&dev)) != Q4_OK) return st;
+    return after_launch(launch_small_m(codes, scales, codebook, x, y, 1, N, K, stream, dev));
+}
+
+q4_status q4_gemm(const uint8_t* codes, const uint16_t* scales, const uint16_t* codebook,
+                  const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
+                  q4_stream_t stream) {
+    bool empty;
+    q4_status st = check_matmul(codes, scales, codebook, x, y, M, N, K, &empty);
+    if (st != Q4_OK || empty) return st;
+    DeviceInfo dev;
+    if ((st = gate(&dev)) != Q4_OK) return st;
+    if (M <= 16)
+        return after_launch(
+            launch_small_m(codes, scales, codebook, x, y, static_cast<int>(M), N, K, stream, dev));
+    return after_launch(launch_prefill(codes, scales, codebook, x, y, M, N, K, stream, dev));
+}
+
+const char* q4_status_string(q4_status status) {
+    switch (status) {
+        case Q4_OK: return "Q4_OK";
+        case Q4_ERR_NULL: return "Q4_ERR_NULL: a required pointer is NULL";
+        case Q4_ERR_SHAPE: return "Q4_ERR_SHAPE: bad M, N or K";
+        case Q4_ERR_ALIGN: return "Q4_ERR_ALIGN: a pointer is not 16-byte aligned";
+        case Q4_ERR_ARCH: return "Q4_ERR_ARCH: the current device is not sm_100";
+        case Q4_ERR_CUDA: return "Q4_ERR_CUDA: a CUDA call or kernel launch failed";
+    }
+    return "unknown q4_status";
+}
+
+int q4_last_cuda_error(void) { return g_last_cuda_error; }
+
+int q4_abi_version(void) { return Q4_ABI_VERSION; }
+
+}  // extern "C"

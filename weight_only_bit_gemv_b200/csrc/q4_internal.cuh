@@ -1,0 +1,100 @@
+// q4_internal.cuh -- internal declarations and device helpers of the sm_100a
+// 4-bit codebook linear-layer library.  Not part of the public ABI (q4.h).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "q4.h"
+
+namespace q4 {
+
+constexpr int kGroup = 64;  // weights per scale group, along K
+
+// ---------------------------------------------------------------------------
+// per-device properties, queried once per device (q4_api.cu)
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+    int device;
+    int sm_count;
+    int cc_major, cc_minor;
+    int smem_optin;  // max dynamic shared memory per block (opt-in)
+};
+// Fills *info for the current device; returns cudaSuccess or the failing code.
+cudaError_t current_device_info(DeviceInfo* info);
+
+// Calls cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per device and
+// kernel; `slot` identifies the kernel (a small dense index per translation
+// unit range, see the launchers).
+cudaError_t ensure_smem_attr(const void* func, int bytes, int slot, int device);
+
+// ---------------------------------------------------------------------------
+// launchers (each validated by q4_api.cu before it is called)
+// ---------------------------------------------------------------------------
+cudaError_t launch_pack(const float* w, const uint16_t* cb, uint8_t* codes, uint16_t* scales,
+                        int64_t N, int64_t K, cudaStream_t s, const DeviceInfo& dev);
+cudaError_t launch_dequant(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                           float* w, int64_t N, int64_t K, cudaStream_t s, const DeviceInfo& dev);
+// M in [1, 16]: decoded codebook values on mma.sync, exact products, fp32 sums.
+cudaError_t launch_small_m(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                           const uint16_t* x, float* y, int M, int64_t N, int64_t K,
+                           cudaStream_t s, const DeviceInfo& dev);
+// M > 16: tcgen05 tensor-core GEMM with TMEM accumulators.
+cudaError_t launch_prefill(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                           const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
+                           cudaStream_t s, const DeviceInfo& dev);
+
+// ---------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint4 lds_u128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+// Streaming 8-byte global load that does not allocate in L1.
+__device__ __forceinline__ uint2 ldg_stream_u2(const void* p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+                 : "=r"(v.x), "=r"(v.y)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint16_t ldg_u16(const void* p) {
+    uint16_t v;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
+// bfloat16 bits -> binary32 (exact)
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
+    return __uint_as_float(b << 16);
+}
+
+// D = A * B + C, m16n8k16, A row-major f16, B column-major f16, fp32 accumulators.
+__device__ __forceinline__ void mma_16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1,
+                                          const float c[4]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1),
+          "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]));
+}
+
+}  // namespace q4
