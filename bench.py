@@ -167,7 +167,8 @@ def capture_graphs(lins, cb, stream, with_events):
     graphs, events = [], []
     for c in range(COPIES):
         g = torch.cuda.CUDAGraph()
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(lins) + 1)] if with_events else []
+        evs = ([torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(lins) + 1)]
+               if with_events else [])
         with torch.cuda.graph(g, stream=stream):
             if with_events:
                 evs[0].record()
