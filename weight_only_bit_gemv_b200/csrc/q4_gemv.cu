@@ -126,9 +126,8 @@ __device__ __forceinline__ void load_stage(Stage<RT, B>& st, const SmallM& p, in
 
 template <int MB, int RT, int B>
 __device__ __forceinline__ void compute_stage(const Stage<RT, B>& st, const SmallM& p, int grp0,
-                                              int ge, int c0, uint32_t lut, uint32_t lane4,
-                                              uint32_t xs, int g, int tq,
-                                              float (&acc)[RT][MB][4]) {
+                                              int ge, int c0, const uint8_t* smem, uint32_t lane4,
+                                              int g, int tq, float (&acc)[RT][MB][4]) {
 #pragma unroll
     for (int j = 0; j < B; ++j) {
         const int gj = grp0 + j;
@@ -139,8 +138,8 @@ __device__ __forceinline__ void compute_stage(const Stage<RT, B>& st, const Smal
         for (int mb = 0; mb < MB; ++mb) {
             const int m = mb * 8 + g;
             if (m < p.M) {
-                const uint32_t a = xs + m * p.pitch + (gj - c0) * 128 + tq * 32;
-                const uint4 v0 = lds_u128(a), v1 = lds_u128(a + 16);
+                const uint32_t a = kLutBytes + m * p.pitch + (gj - c0) * 128 + tq * 32;
+                const uint4 v0 = ld_smem<uint4>(smem, a), v1 = ld_smem<uint4>(smem, a + 16);
                 xb[mb][0] = v0.x; xb[mb][1] = v0.y; xb[mb][2] = v0.z; xb[mb][3] = v0.w;
                 xb[mb][4] = v1.x; xb[mb][5] = v1.y; xb[mb][6] = v1.z; xb[mb][7] = v1.w;
             } else {
@@ -162,15 +161,15 @@ __device__ __forceinline__ void compute_stage(const Stage<RT, B>& st, const Smal
                 const uint32_t wh = (tt < 2) ? hi.x : hi.y;
                 uint32_t a[4];
                 if (tt & 1) {
-                    a[0] = lds_u32(lut + lut_offset<2>(wl, lane4));
-                    a[1] = lds_u32(lut + lut_offset<2>(wh, lane4));
-                    a[2] = lds_u32(lut + lut_offset<3>(wl, lane4));
-                    a[3] = lds_u32(lut + lut_offset<3>(wh, lane4));
+                    a[0] = ld_smem<uint32_t>(smem, lut_offset<2>(wl, lane4));
+                    a[1] = ld_smem<uint32_t>(smem, lut_offset<2>(wh, lane4));
+                    a[2] = ld_smem<uint32_t>(smem, lut_offset<3>(wl, lane4));
+                    a[3] = ld_smem<uint32_t>(smem, lut_offset<3>(wh, lane4));
                 } else {
-                    a[0] = lds_u32(lut + lut_offset<0>(wl, lane4));
-                    a[1] = lds_u32(lut + lut_offset<0>(wh, lane4));
-                    a[2] = lds_u32(lut + lut_offset<1>(wl, lane4));
-                    a[3] = lds_u32(lut + lut_offset<1>(wh, lane4));
+                    a[0] = ld_smem<uint32_t>(smem, lut_offset<0>(wl, lane4));
+                    a[1] = ld_smem<uint32_t>(smem, lut_offset<0>(wh, lane4));
+                    a[2] = ld_smem<uint32_t>(smem, lut_offset<1>(wl, lane4));
+                    a[3] = ld_smem<uint32_t>(smem, lut_offset<1>(wh, lane4));
                 }
 #pragma unroll
                 for (int mb = 0; mb < MB; ++mb)
@@ -236,11 +235,11 @@ __global__ void __launch_bounds__(kThreads, 2) small_m_kernel(const SmallM p) {
             if (grp < ge) load_stage(sa, p, grp, ge, r0, g, tq);
             while (grp < ge) {
                 if (grp + B < ge) load_stage(sb, p, grp + B, ge, r0, g, tq);
-                compute_stage<MB>(sa, p, grp, ge, c0, lut, lane4, xs, g, tq, acc);
+                compute_stage<MB>(sa, p, grp, ge, c0, smem, lane4, g, tq, acc);
                 grp += B;
                 if (grp >= ge) break;
                 if (grp + B < ge) load_stage(sa, p, grp + B, ge, r0, g, tq);
-                compute_stage<MB>(sb, p, grp, ge, c0, lut, lane4, xs, g, tq, acc);
+                compute_stage<MB>(sb, p, grp, ge, c0, smem, lane4, g, tq, acc);
                 grp += B;
             }
         }
@@ -291,6 +290,11 @@ cudaError_t launch_variant(SmallM p, int slot, cudaStream_t s, const DeviceInfo&
 cudaError_t launch_small_m(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int M, int64_t N, int64_t K,
                            cudaStream_t s, const DeviceInfo& dev) {
+    if (M == 1) {
+        cudaError_t e = launch_gemv_tma(codes, scales, cb, x, y, N, K, s, dev);
+        if (e != cudaErrorNotSupported) return e;
+        (void)cudaGetLastError();
+    }
     SmallM p{};
     p.codes = codes;
     p.scales = scales;

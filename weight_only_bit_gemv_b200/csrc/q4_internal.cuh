@@ -40,6 +40,11 @@ cudaError_t launch_dequant(const uint8_t* codes, const uint16_t* scales, const u
 cudaError_t launch_small_m(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int M, int64_t N, int64_t K,
                            cudaStream_t s, const DeviceInfo& dev);
+// M = 1: TMA-fed, warp-specialized decode GEMV.  Returns cudaErrorNotSupported
+// when the shape does not fit it (shared-memory budget).
+cudaError_t launch_gemv_tma(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                            const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
+                            const DeviceInfo& dev);
 // M > 16: tcgen05 tensor-core GEMM with TMEM accumulators.
 cudaError_t launch_prefill(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
@@ -66,19 +71,20 @@ __device__ __forceinline__ uint4 lds_u128(uint32_t addr) {
     return v;
 }
 
-// Streaming 8-byte global load that does not allocate in L1.
+// Streaming 8-byte global load (evict-first); a plain load the compiler can schedule.
 __device__ __forceinline__ uint2 ldg_stream_u2(const void* p) {
-    uint2 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
-                 : "=r"(v.x), "=r"(v.y)
-                 : "l"(p));
-    return v;
+    return __ldcs(reinterpret_cast<const uint2*>(p));
 }
 
 __device__ __forceinline__ uint16_t ldg_u16(const void* p) {
-    uint16_t v;
-    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
-    return v;
+    return __ldg(reinterpret_cast<const unsigned short*>(p));
+}
+
+// Shared-memory loads as plain C++ accesses: ordered after any asm volatile
+// with a memory clobber (the mbarrier waits), otherwise free to be scheduled.
+template <typename T>
+__device__ __forceinline__ T ld_smem(const uint8_t* smem, uint32_t off) {
+    return *reinterpret_cast<const T*>(smem + off);
 }
 
 // bfloat16 bits -> binary32 (exact)
@@ -87,9 +93,11 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
 }
 
 // D = A * B + C, m16n8k16, A row-major f16, B column-major f16, fp32 accumulators.
+// Not volatile: a pure function of its registers, so the compiler may
+// schedule it among the loads that feed it.
 __device__ __forceinline__ void mma_16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1,
                                           const float c[4]) {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
         "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%10, %11, %12, %13};"
         : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
