@@ -46,8 +46,14 @@ __device__ unsigned int g_gemv_tma_error;
 
 namespace {
 
-constexpr int kC = 8;                        // consumer warps
-constexpr int kR = 16 * kC;                  // rows per strip
+// Consumer warps: kTiles 16-row tiles x kHalves.  With two halves, warp
+// (tile, h) decodes groups 4h .. 4h+3 of every stage (one code box each) and
+// the two halves of a tile add up at the end of a strip; measured on B200 it
+// is no faster than one warp per tile, which is the setting used.
+constexpr int kTiles = 8;
+constexpr int kHalves = 1;
+constexpr int kC = kTiles * kHalves;         // consumer warps
+constexpr int kR = 16 * kTiles;              // rows per strip
 constexpr int kSG = 8;                       // groups per stage
 constexpr int kBoxBytes = kR * 128;          // one code box: 4 groups x 128 rows
 constexpr int kCodeStageBytes = 2 * kBoxBytes;
@@ -65,7 +71,7 @@ struct TmaGemv {
     float* y;
     int N, K, G, KS, strips;
     int stages;
-    int scale_off, xs_off, cb_off, bar_off;
+    int scale_off, xs_off, cb_off, pair_off, bar_off;
 };
 
 __device__ __forceinline__ uint32_t cvt_bf16x2_f16x2(uint32_t w) {
@@ -267,7 +273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int g = lane >> 2, tq = lane & 3;
     const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
-    const int r_lo = 16 * warp + 2 * g, r_hi = r_lo + 1;
+    const int tile = warp % kTiles, my_half = warp / kTiles;
+    const int r_lo = 16 * tile + 2 * g, r_hi = r_lo + 1;
     uint32_t off_lo[4], off_hi[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -283,7 +290,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     long long u = u0;
     int strip = static_cast<int>(u / p.KS), ks = static_cast<int>(u % p.KS);
     int cur = strip;
+    float* pair_buf = reinterpret_cast<float*>(smem + p.pair_off) + tile * 32;
     auto flush = [&](int st) {
+        if (kHalves == 2) {
+            // the second half hands its partial sums to the first
+            if (my_half == 1 && tq == 0) {
+                pair_buf[2 * g] = acc_lo;
+                pair_buf[2 * g + 1] = acc_hi;
+            }
+            asm volatile("bar.sync %0, 64;" ::"r"(2 + tile) : "memory");
+            if (my_half == 1) {
+                asm volatile("bar.sync %0, 64;" ::"r"(2 + tile) : "memory");
+                return;
+            }
+            if (tq == 0) {
+                acc_lo += pair_buf[2 * g];
+                acc_hi += pair_buf[2 * g + 1];
+            }
+            asm volatile("bar.sync %0, 64;" ::"r"(2 + tile) : "memory");
+        }
         if (tq != 0) return;
         const bool whole = static_cast<long long>(st) * p.KS >= u0 &&
                            static_cast<long long>(st + 1) * p.KS <= u1;
@@ -315,10 +340,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t soff = p.scale_off + slot * kScaleStageBytes;
         const uint4 sl = ld_smem<uint4>(smem, soff + r_lo * 16);
         const uint4 sh = ld_smem<uint4>(smem, soff + r_hi * 16);
-        const uint32_t slw[4] = {sl.x, sl.y, sl.z, sl.w};
-        const uint32_t shw[4] = {sh.x, sh.y, sh.z, sh.w};
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int hh = 0; hh < 2 / kHalves; ++hh) {
+            const int half = (kHalves == 2) ? my_half : hh;
+            // scale words of this half: groups 4 half .. 4 half + 3
+            const uint32_t sl0 = half ? sl.z : sl.x, sl1 = half ? sl.w : sl.y;
+            const uint32_t sh0 = half ? sh.z : sh.x, sh1 = half ? sh.w : sh.y;
             uint2 clo[4], chi[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -336,9 +363,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 4; ++j) {
                 float d0, d2;
                 group_mma(smem, clo[j], chi[j], xa[j], xb[j], lane4, d0, d2);
-                const int q = 4 * half + j;
-                const float s_lo = (q & 1) ? half_hi(slw[q >> 1]) : half_lo(slw[q >> 1]);
-                const float s_hi = (q & 1) ? half_hi(shw[q >> 1]) : half_lo(shw[q >> 1]);
+                const uint32_t wl = (j < 2) ? sl0 : sl1, wh = (j < 2) ? sh0 : sh1;
+                const float s_lo = (j & 1) ? half_hi(wl) : half_lo(wl);
+                const float s_hi = (j & 1) ? half_hi(wh) : half_lo(wh);
                 acc_lo = fmaf(s_lo, d0, acc_lo);
                 acc_hi = fmaf(s_hi, d2, acc_hi);
             }
@@ -376,7 +403,7 @@ cudaError_t launch_gemv_tma(const uint8_t* codes, const uint16_t* scales, const 
     p.strips = static_cast<int>((N + kR - 1) / kR);
     const int x_bytes = p.KS * kSG * kGroup * 2;
     const int per_stage = kCodeStageBytes + kScaleStageBytes;
-    const int fixed = kLutBytes + x_bytes + 32 + (2 * kMaxStages + 1) * 8 + 1024;
+    const int fixed = kLutBytes + x_bytes + 32 + kTiles * 128 + (2 * kMaxStages + 1) * 8 + 1024;
     int S = (dev.smem_optin - fixed) / per_stage;
     if (S > kMaxStages) S = kMaxStages;
     if (S < 2) return cudaErrorNotSupported;
@@ -384,7 +411,8 @@ cudaError_t launch_gemv_tma(const uint8_t* codes, const uint16_t* scales, const 
     p.scale_off = kLutBytes + S * kCodeStageBytes;
     p.xs_off = p.scale_off + S * kScaleStageBytes;
     p.cb_off = p.xs_off + x_bytes;
-    p.bar_off = p.cb_off + 32;
+    p.pair_off = p.cb_off + 32;
+    p.bar_off = p.pair_off + kTiles * 32 * 4;
     const int smem = p.bar_off + (2 * S + 1) * 8;
 
     const int mode = (p.G % 8 == 0) ? kScaleTma : (p.G % 4 == 0) ? kScaleAsync : kScaleSync;
