@@ -27,8 +27,12 @@
  *   w        float    [N][K]     binary32 (input of q4_pack, output of q4_dequant)
  *
  * Ownership.  Every pointer is device memory owned by the caller (PyTorch,
- * cudaMalloc, ...).  The library allocates nothing, keeps no pointer after a
- * call returns, and holds only a per-device cache of the device's properties.
+ * cudaMalloc, ...).  The library keeps no pointer after a call returns and
+ * holds only a per-device cache of the device's properties.  The one
+ * allocation it makes is the stream-ordered scratch of q4_gemm with M > 16
+ * (2 * M * K bytes for the binary16 copy of x), taken from a memory pool the
+ * library creates once per device and returned to that pool on the same
+ * stream before the call returns; the pool keeps the memory it has mapped.
  * All calls are asynchronous on the caller's stream (0 = legacy default
  * stream); none synchronizes the host.  Inputs and outputs must not overlap.
  * The calls are thread-safe.
@@ -129,6 +133,11 @@ q4_status q4_gemv(const uint8_t* codes, const uint16_t* scales,
  * exact sum per element (for the tensor-core path this holds statistically:
  * the binary16 rounding of W and x is a relative error of at most 2^-11 per
  * term, far inside the bound once K is a few hundred).
+ * M > 16 first converts x to binary16 into stream-ordered scratch (see
+ * Ownership); a failed scratch allocation returns Q4_ERR_CUDA.  When the
+ * K dimension is split across thread blocks, y is zeroed on the stream and
+ * the partial sums are added into it atomically, so the summation order (and
+ * the last bits of y) may vary between runs.
  * In: codes, scales, codebook, x [M][K] bf16.  Out: y [M][N] fp32.
  */
 q4_status q4_gemm(const uint8_t* codes, const uint16_t* scales,
@@ -144,6 +153,18 @@ int q4_last_cuda_error(void);
 
 /* Q4_ABI_VERSION of the library that was loaded. */
 int q4_abi_version(void);
+
+/*
+ * q4_timeout_flags -- every wait inside the TMA and tensor-core kernels is
+ * bounded (about two seconds); a wait that runs out sets a bit in a device
+ * word, the kernel drains what it has in flight, frees its tensor memory and
+ * exits, leaving its output incomplete.  This call synchronizes the current
+ * device, stores the bits set since the last call in *flags (bits 0-15: the
+ * M = 1 TMA GEMV; bits 16-31: the M > 16 tensor-core GEMM; 0 = no timeout)
+ * and clears them.  Not an operation of the method; a health check.
+ * Returns Q4_ERR_NULL for a NULL flags, Q4_ERR_CUDA if a CUDA call fails.
+ */
+q4_status q4_timeout_flags(uint32_t* flags);
 
 #ifdef __cplusplus
 }

@@ -23,7 +23,7 @@ def lib():
 def test_exports_every_declared_function(lib):
     names = q4.header_functions()
     assert {"q4_pack", "q4_dequant", "q4_gemv", "q4_gemm", "q4_status_string",
-            "q4_last_cuda_error", "q4_abi_version"} <= set(names)
+            "q4_last_cuda_error", "q4_abi_version", "q4_timeout_flags"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", q4.library_path()],
                          capture_output=True, text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
@@ -64,6 +64,10 @@ def test_gemm_rejects(lib):
     assert f(A, A, A, MIS, A, 5, 64, 64, None) == ALIGN
     assert f(A, A, A, A, MIS, 5, 64, 64, None) == ALIGN
     assert f(A, A, MIS, A, A, 5, 64, 64, None) == ALIGN
+
+
+def test_timeout_flags_rejects_null(lib):
+    assert lib.q4_timeout_flags(None) == NULL
 
 
 def test_pack_dequant_reject(lib):

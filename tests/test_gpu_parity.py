@@ -153,6 +153,20 @@ def test_integer_codebook_exact(M):
         assert np.array_equal(run_matmul(codes, scales, cb, x, "gemv"), y_ref)
 
 
+@pytest.mark.parametrize("M,N,K", [(40, 300, 64), (300, 130, 640), (257, 64, 1088),
+                                   (20, 1, 256), (512, 129, 192)])
+def test_integer_codebook_exact_prefill_shapes(M, N, K):
+    """Tensor-core tiling edges: one group (no K split), two token tiles,
+    group counts that are not a multiple of four, a single output row."""
+    rng = np.random.default_rng(M * 7 + N + K)
+    cb = synth.integer_codebook()
+    codes = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    scales = np.asarray(2.0 ** rng.integers(0, 3, size=(N, K // GROUP)), np.float16).view(np.uint16)
+    x = synth.f32_to_bf16_bits(rng.integers(-4, 5, size=(M, K)).astype(np.float32))
+    y_ref, _ = oracle.matmul(codes, scales, cb, x)
+    assert np.array_equal(run_matmul(codes, scales, cb, x), y_ref)
+
+
 @pytest.mark.parametrize("M", [1, 5, 16, 33])
 def test_one_hot_selects_column(M):
     N, K = 96, 512
@@ -191,7 +205,8 @@ def test_tiny_config_gemv():
 @pytest.mark.parametrize("M,N,K", [
     (1, 1, 64), (1, 7, 128), (1, 17, 448), (1, 1000, 4160), (1, 33, 28672),
     (3, 100, 192), (8, 129, 1024), (9, 31, 2048), (16, 300, 4096), (16, 64, 14336),
-    (17, 130, 512), (64, 257, 1088), (100, 96, 4096)])
+    (17, 130, 512), (64, 257, 1088), (100, 96, 4096),
+    (300, 200, 640), (257, 130, 2048), (48, 1000, 4160)])
 def test_ragged_shapes(M, N, K):
     codes, scales = random_packed(M * 1000 + N, N, K)
     x = synth.activations(K + N, M, K)
@@ -273,3 +288,8 @@ def test_llama2_70b_prefill(linear, M):
     assert np.all(np.isfinite(y))
     rows = np.random.default_rng(M + 1).choice(codes.shape[0], size=256, replace=False)
     assert_close(y, codes, scales, NF4, x, rows=rows, label=f"{linear} M={M}")
+
+
+def test_no_bounded_wait_ran_out():
+    """Collected last in this file: no kernel above gave up on a wait."""
+    assert q4.timeout_flags() == 0

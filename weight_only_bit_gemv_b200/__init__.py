@@ -68,6 +68,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.q4_last_cuda_error.restype = ctypes.c_int
     lib.q4_abi_version.argtypes = []
     lib.q4_abi_version.restype = ctypes.c_int
+    lib.q4_timeout_flags.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+    lib.q4_timeout_flags.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -182,6 +184,13 @@ def q4_gemv(codes, scales, codebook, x, y=None, stream=None) -> torch.Tensor:
 def q4_gemm(codes, scales, codebook, x, y=None, stream=None) -> torch.Tensor:
     """y [M, N] = x [M, K] @ W^T for any M (M <= 16: verify batches; M > 16: prefill)."""
     return _matmul("q4_gemm", codes, scales, codebook, x, y, stream)
+
+
+def timeout_flags() -> int:
+    """Synchronize the current device; return and clear the kernels' bounded-wait timeout bits."""
+    out = ctypes.c_uint32(0)
+    _check(load().q4_timeout_flags(ctypes.byref(out)), "q4_timeout_flags")
+    return int(out.value)
 
 
 def abi_version() -> int:

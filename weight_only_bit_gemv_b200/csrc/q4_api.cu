@@ -188,4 +188,15 @@ int q4_last_cuda_error(void) { return g_last_cuda_error; }
 
 int q4_abi_version(void) { return Q4_ABI_VERSION; }
 
+q4_status q4_timeout_flags(uint32_t* flags) {
+    if (!flags) return Q4_ERR_NULL;
+    *flags = 0;
+    unsigned int a = 0, b = 0;
+    cudaError_t e = take_gemv_tma_error(&a);
+    if (e == cudaSuccess) e = take_gemm_tc_error(&b);
+    if (e != cudaSuccess) return cuda_fail(e);
+    *flags = (a & 0xFFFFu) | ((b & 0xFFFFu) << 16);
+    return Q4_OK;
+}
+
 }  // extern "C"

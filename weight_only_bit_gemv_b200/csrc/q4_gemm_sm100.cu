@@ -1,17 +1,507 @@
-// q4_gemm_sm100.cu -- q4_gemm for M > 16.
+// q4_gemm_sm100.cu -- q4_gemm for M > 16 (prompt processing): a tcgen05
+// tensor-core GEMM whose A operand is rebuilt from the 4-bit codes straight
+// into tensor memory.
+//
+// What it computes: y[m][n] = sum_k W[n][k] x[m][k] with W[n][k] =
+// cb[code(n,k)] * scale[n][k/64] ("deep-fold", "Method" table: prompt
+// processing runs a tensor-core NF4 GEMM that rebuilds weights into
+// fragments while it multiplies; no dense weight matrix is written).
+//
+// Numerics: each weight is rebuilt as binary16(cb * scale) -- HMUL2 of two
+// binary16 values, one rounding of the exact product -- and x is rounded to
+// binary16 once (exact for 2^-17 <= |x| <= 65504).  Products accumulate in
+// fp32 in tensor memory.  The per-weight relative error is at most 2^-11,
+// which keeps every output inside 1e-4 * sum|W x| + 1e-6 with a margin of
+// ~0.3 sqrt(K) standard deviations (about 20 at K = 4096).
+//
+// Roles (one CTA per tile of 128 weight rows x BMT tokens x one K chunk):
+//  * warp 0 streams, by TMA, stages of 4 groups of codes (a 128-row x
+//    128-byte box, 128-byte swizzle) with their scales (cp.async), and for
+//    every group the x tile (BMT tokens x 64 k binary16, 128-byte swizzle).
+//  * warps 2-9 rebuild the weights: thread t of warp w owns row 32 (w mod 4) +
+//    t (its tensor-memory lane); per group it reads its 32 code bytes, looks
+//    each up in a 256-entry byte -> (cb[lo], cb[hi]) table (one copy per
+//    lane), multiplies by the scale with one HMUL2 and writes the 64 weights
+//    with one tcgen05.st into one of four A slots.  Even and odd groups go to
+//    the two halves of these warps.
+//  * warp 1 owns the tensor memory and, per group, issues four tcgen05.mma
+//    M=128 N=BMT K=16 (A from tensor memory, B = x tile from shared memory)
+//    into one fp32 accumulator of BMT columns; commits free the A slot and
+//    the x slot, and a last commit marks the accumulator ready.
+//  * warps 2-9 then read the accumulator (tcgen05.ld) and write y, or add it
+//    into y with red.add when K is split across CTAs (y zeroed first).
+// Every wait is bounded; a timeout sets an error bit, the roles drain what
+// they have in flight and the CTA frees its tensor memory before it exits.
+#include <mutex>
+
 #include "q4_internal.cuh"
+#include "q4_sm100.cuh"
 
 namespace q4 {
+
+__device__ unsigned int g_gemm_tc_error;
+
+namespace {
+
+constexpr int kR = 128;                   // weight rows per tile = tensor-memory lanes
+constexpr int kWG = 4;                    // groups per weight stage
+constexpr int kWCodeBytes = kR * 128;     // one code box
+constexpr int kWScaleBytes = kR * 8;      // 4 scales per row
+constexpr int kLutBytes = 65536;
+constexpr int kDecWarps = 8;
+constexpr int kThreads = (2 + kDecWarps) * 32;
+constexpr int kASlots = 4;
+constexpr int kWStages = 3;
+constexpr uint32_t kTmemCols = 512;
+__device__ __forceinline__ uint32_t a_col(int slot) { return 256u + 32u * slot; }
+
+struct TcGemm {
+    const uint16_t* scales;
+    const uint16_t* cb;
+    float* y;
+    int M, N, K, G;
+    int BMT;            // tokens per tile (MMA N), multiple of 16, <= 256
+    int token_tiles;    // ceil(M / BMT)
+    int ksplit;         // K chunks per tile
+    int chunk_groups;   // groups per K chunk (multiple of kWG)
+    int xstages;
+    int xstage_bytes;   // BMT * 128
+    int wscale_off, x_off, cb_off, bar_off;
+    uint32_t idesc;
+};
+
+__device__ __forceinline__ void named_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int lane) {
+    uint32_t ok = 1;
+    if (lane == 0) ok = mbar_wait(bar, parity) ? 1u : 0u;
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+template <int kByte>
+__device__ __forceinline__ uint32_t lut_at(const uint8_t* smem, uint32_t word, uint32_t lane4) {
+    return ld_smem<uint32_t>(smem, __byte_perm(word, lane4, 0x5504 | (kByte << 4)));
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+    __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+    return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+template <bool kAsyncScales>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap xmap,
+                   const TcGemm p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bars = base + p.bar_off;
+    const int SX = p.xstages;
+    // barriers: wfull[2], wempty[2], xfull[SX], xempty[SX], afull[4], afree[4], dfull, cbbar, drain
+    auto wfull = [&](int s) { return bars + 8u * s; };
+    auto wempty = [&](int s) { return bars + 8u * (kWStages + s); };
+    auto xfull = [&](int s) { return bars + 8u * (2 * kWStages + s); };
+    auto xempty = [&](int s) { return bars + 8u * (2 * kWStages + SX + s); };
+    auto afull = [&](int s) { return bars + 8u * (2 * kWStages + 2 * SX + s); };
+    auto afree = [&](int s) { return bars + 8u * (2 * kWStages + 2 * SX + kASlots + s); };
+    const uint32_t dfull = bars + 8u * (2 * kWStages + 2 * SX + 2 * kASlots);
+    const uint32_t cbbar = dfull + 8u;
+    const uint32_t drain = dfull + 16u;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + p.cb_off + 32);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + p.cb_off + 36);
+
+    // tile coordinates: blockIdx.x = ((strip * token_tiles) + tt) * ksplit + kc
+    const int kc = blockIdx.x % p.ksplit;
+    const int tt = (blockIdx.x / p.ksplit) % p.token_tiles;
+    const int strip = blockIdx.x / (p.ksplit * p.token_tiles);
+    const int g_begin = kc * p.chunk_groups;
+    const int g_end = min(p.G, g_begin + p.chunk_groups);
+    const int ng = g_end - g_begin;  // groups of this CTA, >= 1
+    const int nw = (ng + kWG - 1) / kWG;
+
+    if (tid == 0) {
+        for (int s = 0; s < kWStages; ++s) {
+            mbar_init(wfull(s), 33);  // expect_tx + one arrival per producer lane
+            mbar_init(wempty(s), kDecWarps);
+        }
+        for (int s = 0; s < SX; ++s) {
+            mbar_init(xfull(s), 1);
+            mbar_init(xempty(s), 1);  // tcgen05.commit
+        }
+        for (int s = 0; s < kASlots; ++s) {
+            mbar_init(afull(s), 4);   // the four warps of the owning warpgroup
+            mbar_init(afree(s), 1);   // tcgen05.commit
+        }
+        mbar_init(dfull, 1);
+        mbar_init(cbbar, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(base + p.cb_off + 32, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------ producer ------------------------------
+        if (lane == 0) {
+            prefetch_tensor_map(&cmap);
+            prefetch_tensor_map(&xmap);
+            mbar_arrive_expect_tx(cbbar, 32u);
+            bulk_load(base + p.cb_off, p.cb, 32u, cbbar);
+        }
+        int wi = 0, xi = 0;  // weight stages and x tiles issued
+        bool ok = true;
+        for (int w = 0; w < nw && ok; ++w) {
+            // weight stage w: groups g_begin + 4w .. +3
+            const int ws = w % kWStages;
+            if (w >= kWStages && !warp_wait(wempty(ws), static_cast<uint32_t>(w / kWStages - 1) & 1u, lane)) {
+                ok = false;
+                break;
+            }
+            const int g0 = g_begin + kWG * w;
+            const uint32_t cdst = base + kLutBytes + ws * kWCodeBytes;
+            const uint32_t sdst = base + p.wscale_off + ws * kWScaleBytes;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(wfull(ws), kWCodeBytes);
+                tma_load_2d(cdst, &cmap, g0 * 32, strip * kR, wfull(ws));
+            }
+#pragma unroll
+            for (int jr = 0; jr < kR / 32; ++jr) {
+                const int r = lane + 32 * jr;
+                const int row = strip * kR + r;
+                if (kAsyncScales) {
+                    const bool in = row < p.N;
+                    const uint16_t* src = in ? p.scales + static_cast<long long>(row) * p.G + g0 : p.scales;
+                    cp_async_8(sdst + r * 8, src, in ? 8u : 0u);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < kWG; ++q) {
+                        uint16_t v = 0;
+                        if (row < p.N && g0 + q < g_end)
+                            v = p.scales[static_cast<long long>(row) * p.G + g0 + q];
+                        sts_u16(sdst + r * 8 + 2 * q, v);
+                    }
+                }
+            }
+            if (kAsyncScales)
+                cp_async_arrive_noinc(wfull(ws));
+            else
+                mbar_arrive(wfull(ws));
+            ++wi;
+            // x tiles of these groups
+            for (int j = 0; j < kWG && ok; ++j) {
+                const int g = g0 + j;
+                if (g >= g_end) break;
+                const int xs = xi % SX;
+                if (xi >= SX && !warp_wait(xempty(xs), static_cast<uint32_t>(xi / SX - 1) & 1u, lane)) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(xfull(xs), static_cast<uint32_t>(p.xstage_bytes));
+                    tma_load_2d(base + p.x_off + xs * p.xstage_bytes, &xmap, g * 64, tt * p.BMT, xfull(xs));
+                }
+                __syncwarp();
+                ++xi;
+            }
+        }
+        if (!ok && lane == 0) {
+            atomicOr(&g_gemm_tc_error, 1u);
+            *abort_flag = 1;
+        }
+        // leave only once every copy issued has landed (bounded)
+        for (int i = (wi > kWStages ? wi - kWStages : 0); i < wi; ++i)
+            if (!warp_wait(wfull(i % kWStages), static_cast<uint32_t>(i / kWStages) & 1u, lane)) break;
+        for (int i = (xi > SX ? xi - SX : 0); i < xi; ++i)
+            if (!warp_wait(xfull(i % SX), static_cast<uint32_t>(i / SX) & 1u, lane)) break;
+    } else if (warp == 1) {
+        // -------------------------------- MMA ---------------------------------
+        if (lane == 0) {
+            bool ok = true;
+            for (int gi = 0; gi < ng && ok; ++gi) {
+                const int as = gi % kASlots, xs = gi % SX;
+                if (!mbar_wait(afull(as), static_cast<uint32_t>(gi / kASlots) & 1u) ||
+                    !mbar_wait(xfull(xs), static_cast<uint32_t>(gi / SX) & 1u) || *abort_flag) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t bd = smem_desc_sw128(base + p.x_off + xs * p.xstage_bytes, 1024);
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                    tc_mma_ts(tmem, tmem + a_col(as) + 8 * t, bd + 2 * t, p.idesc, (gi > 0 || t > 0) ? 1u : 0u);
+                tc_commit(afree(as));
+                tc_commit(xempty(xs));
+            }
+            if (ok) tc_commit(dfull);
+            if (!ok) {
+                atomicOr(&g_gemm_tc_error, 2u);
+                *abort_flag = 1;
+            }
+            tc_commit(drain);
+            if (!mbar_wait(drain, 0u)) atomicOr(&g_gemm_tc_error, 16u);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------ decoders -------------------------------
+        const int dw = warp - 2, wg = dw >> 2, q = warp & 3;
+        const int row = 32 * q + lane;
+        const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+        const uint32_t tlane = tmem + (static_cast<uint32_t>(32 * q) << 16);
+        bool ok = warp_wait(cbbar, 0u, lane);
+        if (ok) {
+            const uint32_t cbv = ld_smem<uint16_t>(smem, p.cb_off + 2 * (lane & 15));
+            for (int b = dw; b < 256; b += kDecWarps) {
+                const uint32_t lo = __shfl_sync(0xFFFFFFFFu, cbv, b & 15);
+                const uint32_t hi = __shfl_sync(0xFFFFFFFFu, cbv, b >> 4);
+                *reinterpret_cast<uint32_t*>(smem + b * 256 + lane * 4) = lo | (hi << 16);
+            }
+        }
+        named_sync(2, kDecWarps * 32);  // table ready
+
+        // warpgroup wg decodes groups gi = wg, wg + 2, ... into A slots gi mod 4
+        for (int gi = wg; gi < ng && ok; gi += 2) {
+            const int w = gi / kWG, ws = w % kWStages, j = gi % kWG;
+            const int as = gi % kASlots;
+            if (!warp_wait(wfull(ws), static_cast<uint32_t>(w / kWStages) & 1u, lane) ||
+                __shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) {
+                ok = false;
+                break;
+            }
+            if (gi >= kASlots && !warp_wait(afree(as), static_cast<uint32_t>(gi / kASlots - 1) & 1u, lane)) {
+                ok = false;
+                break;
+            }
+            const uint32_t rb = kLutBytes + ws * kWCodeBytes + row * 128;
+            const int r8 = row & 7;
+            const uint4 c0 = ld_smem<uint4>(smem, rb + (((2 * j) ^ r8) << 4));
+            const uint4 c1 = ld_smem<uint4>(smem, rb + (((2 * j + 1) ^ r8) << 4));
+            const uint32_t sb = ld_smem<uint16_t>(smem, p.wscale_off + ws * kWScaleBytes + row * 8 + 2 * j);
+            const uint32_t s2 = sb | (sb << 16);
+            const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            uint32_t h[32];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                h[4 * i + 0] = hmul2_u32(lut_at<0>(smem, wd[i], lane4), s2);
+                h[4 * i + 1] = hmul2_u32(lut_at<1>(smem, wd[i], lane4), s2);
+                h[4 * i + 2] = hmul2_u32(lut_at<2>(smem, wd[i], lane4), s2);
+                h[4 * i + 3] = hmul2_u32(lut_at<3>(smem, wd[i], lane4), s2);
+            }
+            tc_st_x32(tlane + a_col(as), h);
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(afull(as));
+            // this warpgroup's last group of the weight stage releases it
+            const bool last_in_stage = (j + 2 >= kWG) || (gi + 2 >= ng);
+            if (last_in_stage) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(wempty(ws));
+            }
+        }
+        if (!ok && lane == 0) {
+            atomicOr(&g_gemm_tc_error, 8u);
+            *abort_flag = 1;
+        }
+        // epilogue: each warpgroup writes half of the accumulator columns
+        if (warp_wait(dfull, 0u, lane)) {
+            tc_fence_after();
+            const int n = strip * kR + row;
+            const int half = p.BMT / 2;
+            for (int c0 = wg * half; c0 < (wg + 1) * half; c0 += 8) {
+                uint32_t v[8];
+                asm volatile(
+                    "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                    : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                      "=r"(v[7])
+                    : "r"(tlane + c0)
+                    : "memory");
+                tc_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int m = tt * p.BMT + c0 + e;
+                    if (n < p.N && m < p.M) {
+                        float* dst = p.y + static_cast<long long>(m) * p.N + n;
+                        if (p.ksplit > 1)
+                            red_add_f32(dst, __uint_as_float(v[e]));
+                        else
+                            *dst = __uint_as_float(v[e]);
+                    }
+                }
+            }
+        } else if (lane == 0) {
+            atomicOr(&g_gemm_tc_error, 32u);
+        }
+    }
+
+    // -------------------------------- teardown --------------------------------
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+__global__ void bf16_to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xh, int64_t n8) {
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + i);
+        uint4 h;
+        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+        uint32_t out[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const __half2 t = __floats2half2_rn(__uint_as_float(in[q] << 16),
+                                                __uint_as_float(in[q] & 0xFFFF0000u));
+            out[q] = *reinterpret_cast<const uint32_t*>(&t);
+        }
+        h.x = out[0];
+        h.y = out[1];
+        h.z = out[2];
+        h.w = out[3];
+        reinterpret_cast<uint4*>(xh)[i] = h;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_tc(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                              const uint16_t* x, uint16_t* xh, float* y, int64_t M, int64_t N,
+                              int64_t K, cudaStream_t s, const DeviceInfo& dev) {
+    TcGemm p{};
+    p.scales = scales;
+    p.cb = cb;
+    p.y = y;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.G = static_cast<int>(K / kGroup);
+    // token tiles of at most 256 (the largest MMA N), balanced, multiples of 16
+    p.token_tiles = static_cast<int>((M + 255) / 256);
+    p.BMT = static_cast<int>(((M + p.token_tiles - 1) / p.token_tiles + 15) / 16 * 16);
+    const int strips = static_cast<int>((N + kR - 1) / kR);
+    const int tiles = strips * p.token_tiles;
+    // K split: fewest waves x longest chunk (plus a fixed cost of ~4 groups),
+    // one CTA per SM; ties go to the smaller split
+    int ksplit = 1, chunk = (p.G + kWG - 1) / kWG * kWG;
+    long long best = -1;
+    for (int ks = 1; ks <= (p.G + kWG - 1) / kWG; ++ks) {
+        const int c = ((p.G + ks - 1) / ks + kWG - 1) / kWG * kWG;
+        const int real = (p.G + c - 1) / c;
+        if (real != ks) continue;
+        const long long waves = (static_cast<long long>(tiles) * ks + dev.sm_count - 1) / dev.sm_count;
+        const long long cost = waves * (c + 4);
+        if (best < 0 || cost < best) {
+            best = cost;
+            ksplit = ks;
+            chunk = c;
+        }
+    }
+    p.ksplit = ksplit;
+    p.chunk_groups = chunk;
+    p.xstage_bytes = p.BMT * 128;
+    p.idesc = idesc_f16_f32(kR, p.BMT);
+    p.wscale_off = kLutBytes + kWStages * kWCodeBytes;
+    p.x_off = (p.wscale_off + kWStages * kWScaleBytes + 1023) & ~1023;
+    const int fixed = p.x_off + 64 + 512 + 1024;
+    int SX = (dev.smem_optin - fixed) / p.xstage_bytes;
+    if (SX > 6) SX = 6;
+    if (SX < 2) return cudaErrorNotSupported;
+    p.xstages = SX;
+    p.cb_off = p.x_off + SX * p.xstage_bytes;
+    p.bar_off = p.cb_off + 64;
+    const int nbars = 2 * kWStages + 2 * SX + 2 * kASlots + 3;
+    const int smem = p.bar_off + nbars * 8;
+
+    // x -> binary16 into the scratch buffer
+    const int64_t n8 = M * K / 8;
+    int cgrid = static_cast<int>((n8 + 255) / 256);
+    if (cgrid > dev.sm_count * 8) cgrid = dev.sm_count * 8;
+    bf16_to_f16_kernel<<<cgrid, 256, 0, s>>>(x, xh, n8);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    CUtensorMap cmap, xmap;
+    e = encode_tensor_map_2d(&cmap, codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(N),
+                             static_cast<uint64_t>(K / 2), static_cast<uint64_t>(K / 2), kR, 128,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    e = encode_tensor_map_2d(&xmap, xh, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, static_cast<uint64_t>(M),
+                             static_cast<uint64_t>(K), static_cast<uint64_t>(K) * 2, p.BMT, 64,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    if (ksplit > 1) {
+        e = cudaMemsetAsync(y, 0, static_cast<size_t>(M) * N * sizeof(float), s);
+        if (e != cudaSuccess) return e;
+    }
+    const bool async_scales = (p.G % kWG) == 0;
+    const void* fn = async_scales ? reinterpret_cast<const void*>(gemm_tc_kernel<true>)
+                                  : reinterpret_cast<const void*>(gemm_tc_kernel<false>);
+    e = ensure_smem_attr(fn, smem, 30 + (async_scales ? 0 : 1), dev.device);
+    if (e != cudaSuccess) return e;
+    const int grid = tiles * ksplit;
+    if (async_scales)
+        gemm_tc_kernel<true><<<grid, kThreads, smem, s>>>(cmap, xmap, p);
+    else
+        gemm_tc_kernel<false><<<grid, kThreads, smem, s>>>(cmap, xmap, p);
+    return cudaGetLastError();
+}
+
+// Stream-ordered scratch for the binary16 copy of x: one pool per device that
+// keeps what it has mapped (release threshold: never), so steady-state calls
+// neither map memory nor synchronize.
+static cudaError_t scratch_pool(int device, cudaMemPool_t* out) {
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!pools[device]) {
+        cudaMemPoolProps props{};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = device;
+        cudaMemPool_t pool;
+        cudaError_t e = cudaMemPoolCreate(&pool, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = ~0ull;
+        e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) return e;
+        pools[device] = pool;
+    }
+    *out = pools[device];
+    return cudaSuccess;
+}
+
+cudaError_t take_gemm_tc_error(unsigned int* out) {
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_gemm_tc_error, sizeof(unsigned int));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_gemm_tc_error, &zero, sizeof(unsigned int));
+    return e;
+}
 
 cudaError_t launch_prefill(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
                            cudaStream_t s, const DeviceInfo& dev) {
-    for (int64_t m0 = 0; m0 < M; m0 += 16) {
-        const int mc = static_cast<int>(M - m0 < 16 ? M - m0 : 16);
-        cudaError_t e = launch_small_m(codes, scales, cb, x + m0 * K, y + m0 * N, mc, N, K, s, dev);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
+    cudaMemPool_t pool;
+    cudaError_t e = scratch_pool(dev.device, &pool);
+    if (e != cudaSuccess) return e;
+    void* xh = nullptr;
+    e = cudaMallocFromPoolAsync(&xh, static_cast<size_t>(M) * K * sizeof(uint16_t), pool, s);
+    if (e != cudaSuccess) return e;
+    e = launch_prefill_tc(codes, scales, cb, x, static_cast<uint16_t*>(xh), y, M, N, K, s, dev);
+    const cudaError_t f = cudaFreeAsync(xh, s);
+    return e != cudaSuccess ? e : f;
 }
 
 }  // namespace q4

@@ -388,6 +388,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Returns cudaErrorNotSupported when the shape does not fit this kernel (the
 // caller then uses the general small-M kernel).
+cudaError_t take_gemv_tma_error(unsigned int* out) {
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_gemv_tma_error, sizeof(unsigned int));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_gemv_tma_error, &zero, sizeof(unsigned int));
+    return e;
+}
+
 cudaError_t launch_gemv_tma(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                             const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
                             const DeviceInfo& dev) {

@@ -50,6 +50,11 @@ cudaError_t launch_prefill(const uint8_t* codes, const uint16_t* scales, const u
                            const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
                            cudaStream_t s, const DeviceInfo& dev);
 
+// Copy out and clear the timeout bits that a kernel family's bounded waits
+// set (synchronous; see q4_timeout_flags).
+cudaError_t take_gemv_tma_error(unsigned int* out);
+cudaError_t take_gemm_tc_error(unsigned int* out);
+
 // ---------------------------------------------------------------------------
 // device helpers
 // ---------------------------------------------------------------------------
