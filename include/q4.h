@@ -72,13 +72,16 @@ typedef enum {
     Q4_ERR_SHAPE = 2,
     Q4_ERR_ALIGN = 3,
     Q4_ERR_ARCH = 4,
-    Q4_ERR_CUDA = 5
+    Q4_ERR_CUDA = 5,
+    Q4_ERR_TOO_LARGE = 6  /* q4_gemm_noalloc only: x does not fit its fixed scratch */
 } q4_status;
 
 #define Q4_ABI_VERSION 1
 #define Q4_GROUP 64
 #define Q4_MAX_K (1 << 20)
 #define Q4_MAX_MN 2147483647LL
+/* Size of the fixed device scratch of q4_gemm_noalloc: 8 MiB per GPU. */
+#define Q4_NOALLOC_SCRATCH_BYTES (8u << 20)
 
 /*
  * q4_pack -- quantize a dense binary32 W [N][K] into codes and scales.
@@ -143,6 +146,39 @@ q4_status q4_gemv(const uint8_t* codes, const uint16_t* scales,
 q4_status q4_gemm(const uint8_t* codes, const uint16_t* scales,
                   const uint16_t* codebook, const uint16_t* x, float* y,
                   int64_t M, int64_t N, int64_t K, q4_stream_t stream);
+
+/*
+ * q4_gemm_noalloc -- q4_gemm for callers that may not allocate device memory.
+ * The paper has no counterpart; this entry point exists for deployment.
+ *
+ * q4_gemm with M > 16 takes 2 * M * K bytes of scratch from a memory pool
+ * (see Ownership).  Some callers cannot let a library do that: engines that
+ * reserve all device memory at start-up for a fixed arena and a KV cache
+ * leave no headroom for a pool that grows later, and hosts that account for
+ * every byte themselves forbid hidden allocations.  This call computes the
+ * same y with the same kernels, but keeps the binary16 copy of x in one
+ * static device array of Q4_NOALLOC_SCRATCH_BYTES (8 MiB), which every GPU
+ * that loads the library holds until the process exits.  It calls no
+ * cudaMalloc, cudaFree or pool routine.
+ *
+ * Limits and hazards:
+ *   - M > 16 needs 2 * M * K <= Q4_NOALLOC_SCRATCH_BYTES (e.g. M = 512 at
+ *     K = 8192); larger inputs return Q4_ERR_TOO_LARGE before anything runs.
+ *     M <= 16 uses no scratch and has no such limit.
+ *   - The array is shared by every call on a device and is not cleared
+ *     between calls (each call overwrites what it reads).  Calls whose work
+ *     can overlap on the GPU -- different streams, or different host threads
+ *     -- race on it and may return wrong results; serialize them.
+ *   - The first call with M > 16 on a device looks up the array's device
+ *     address (a CUDA runtime query, no allocation) with that device
+ *     current; make that first call before any stream capture.
+ * Validation order: Q4_ERR_SHAPE, Q4_ERR_NULL, Q4_ERR_ALIGN (as q4_gemm), then
+ * Q4_ERR_TOO_LARGE, Q4_ERR_ARCH, Q4_ERR_CUDA.
+ * In and out: as q4_gemm.
+ */
+q4_status q4_gemm_noalloc(const uint8_t* codes, const uint16_t* scales,
+                          const uint16_t* codebook, const uint16_t* x, float* y,
+                          int64_t M, int64_t N, int64_t K, q4_stream_t stream);
 
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* q4_status_string(q4_status status);

@@ -23,7 +23,8 @@ def lib():
 def test_exports_every_declared_function(lib):
     names = q4.header_functions()
     assert {"q4_pack", "q4_dequant", "q4_gemv", "q4_gemm", "q4_status_string",
-            "q4_last_cuda_error", "q4_abi_version", "q4_timeout_flags"} <= set(names)
+            "q4_last_cuda_error", "q4_abi_version", "q4_timeout_flags",
+            "q4_gemm_noalloc"} <= set(names)
     out = subprocess.run(["nm", "-D", "--defined-only", q4.library_path()],
                          capture_output=True, text=True, check=True).stdout
     exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
@@ -35,7 +36,7 @@ def test_exports_every_declared_function(lib):
 
 def test_abi_version_and_strings(lib):
     assert q4.abi_version() == 1
-    for code in range(6):
+    for code in range(7):
         s = q4.status_string(code)
         assert s.startswith(q4.STATUS[code])
     assert "unknown" in q4.status_string(99)
@@ -64,6 +65,17 @@ def test_gemm_rejects(lib):
     assert f(A, A, A, MIS, A, 5, 64, 64, None) == ALIGN
     assert f(A, A, A, A, MIS, 5, 64, 64, None) == ALIGN
     assert f(A, A, MIS, A, A, 5, 64, 64, None) == ALIGN
+
+
+def test_gemm_noalloc_rejects(lib):
+    f = lib.q4_gemm_noalloc
+    K = 4096
+    too_many = (8 << 20) // (2 * K) + 1          # one token past the fixed scratch
+    assert f(A, A, A, A, A, too_many, 64, K, None) == 6   # Q4_ERR_TOO_LARGE
+    assert f(A, A, A, A, A, -1, 64, K, None) == SHAPE
+    assert f(None, A, A, A, A, too_many, 64, K, None) == NULL
+    assert f(A, A, A, MIS, A, too_many, 64, K, None) == ALIGN
+    assert f(A, A, A, A, A, 0, 64, K, None) == OK
 
 
 def test_timeout_flags_rejects_null(lib):

@@ -28,7 +28,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "q4.h")
 
 STATUS = {0: "Q4_OK", 1: "Q4_ERR_NULL", 2: "Q4_ERR_SHAPE", 3: "Q4_ERR_ALIGN", 4: "Q4_ERR_ARCH",
-          5: "Q4_ERR_CUDA"}
+          5: "Q4_ERR_CUDA", 6: "Q4_ERR_TOO_LARGE"}
 
 
 class Q4Error(RuntimeError):
@@ -60,7 +60,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.q4_dequant.argtypes = [P, P, P, P, I64, I64, S]
     lib.q4_gemv.argtypes = [P, P, P, P, P, I64, I64, I64, S]
     lib.q4_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, S]
-    for f in ("q4_pack", "q4_dequant", "q4_gemv", "q4_gemm"):
+    lib.q4_gemm_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, S]
+    for f in ("q4_pack", "q4_dequant", "q4_gemv", "q4_gemm", "q4_gemm_noalloc"):
         getattr(lib, f).restype = ctypes.c_int
     lib.q4_status_string.argtypes = [ctypes.c_int]
     lib.q4_status_string.restype = ctypes.c_char_p
@@ -184,6 +185,16 @@ def q4_gemv(codes, scales, codebook, x, y=None, stream=None) -> torch.Tensor:
 def q4_gemm(codes, scales, codebook, x, y=None, stream=None) -> torch.Tensor:
     """y [M, N] = x [M, K] @ W^T for any M (M <= 16: verify batches; M > 16: prefill)."""
     return _matmul("q4_gemm", codes, scales, codebook, x, y, stream)
+
+
+def q4_gemm_noalloc(codes, scales, codebook, x, y, stream=None) -> torch.Tensor:
+    """q4_gemm without any device allocation by the library: for M > 16 the
+    binary16 copy of x lives in the library's fixed 8 MiB device array, so
+    2 * M * K must fit in it (else Q4Error Q4_ERR_TOO_LARGE), and calls that
+    overlap on the GPU race on that array.  y must be passed in."""
+    if y is None:
+        raise ValueError("q4_gemm_noalloc writes into a caller-provided y")
+    return _matmul("q4_gemm_noalloc", codes, scales, codebook, x, y, stream)
 
 
 def timeout_flags() -> int:

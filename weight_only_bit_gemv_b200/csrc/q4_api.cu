@@ -172,6 +172,23 @@ q4_status q4_gemm(const uint8_t* codes, const uint16_t* scales, const uint16_t* 
     return after_launch(launch_prefill(codes, scales, codebook, x, y, M, N, K, stream, dev));
 }
 
+q4_status q4_gemm_noalloc(const uint8_t* codes, const uint16_t* scales, const uint16_t* codebook,
+                          const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
+                          q4_stream_t stream) {
+    bool empty;
+    q4_status st = check_matmul(codes, scales, codebook, x, y, M, N, K, &empty);
+    if (st != Q4_OK || empty) return st;
+    if (M > 16 && static_cast<uint64_t>(M) * static_cast<uint64_t>(K) * sizeof(uint16_t) >
+                      Q4_NOALLOC_SCRATCH_BYTES)
+        return Q4_ERR_TOO_LARGE;
+    DeviceInfo dev;
+    if ((st = gate(&dev)) != Q4_OK) return st;
+    if (M <= 16)
+        return after_launch(
+            launch_small_m(codes, scales, codebook, x, y, static_cast<int>(M), N, K, stream, dev));
+    return after_launch(launch_prefill_noalloc(codes, scales, codebook, x, y, M, N, K, stream, dev));
+}
+
 const char* q4_status_string(q4_status status) {
     switch (status) {
         case Q4_OK: return "Q4_OK";
@@ -180,6 +197,8 @@ const char* q4_status_string(q4_status status) {
         case Q4_ERR_ALIGN: return "Q4_ERR_ALIGN: a pointer is not 16-byte aligned";
         case Q4_ERR_ARCH: return "Q4_ERR_ARCH: the current device is not sm_100";
         case Q4_ERR_CUDA: return "Q4_ERR_CUDA: a CUDA call or kernel launch failed";
+        case Q4_ERR_TOO_LARGE:
+            return "Q4_ERR_TOO_LARGE: 2 * M * K bytes exceed Q4_NOALLOC_SCRATCH_BYTES (q4_gemm_noalloc)";
     }
     return "unknown q4_status";
 }

@@ -504,4 +504,43 @@ cudaError_t launch_prefill(const uint8_t* codes, const uint16_t* scales, const u
     return e != cudaSuccess ? e : f;
 }
 
+// ---------------------------------------------------------------------------
+// q4_gemm_noalloc: the same tensor-core path with its x scratch in a fixed
+// device array instead of the pool, for callers that may not allocate.
+// ---------------------------------------------------------------------------
+// Every GPU that loads the library holds this array until the process exits.
+// All calls share it and it keeps the last call's contents; the conversion
+// kernel overwrites the M * K elements a call reads before the GEMM reads
+// them, so nothing in it has to start at zero.  Calls whose work overlaps on
+// the GPU (other streams, other host threads) race on it.
+static __device__ __align__(256) uint16_t g_noalloc_x[Q4_NOALLOC_SCRATCH_BYTES / sizeof(uint16_t)];
+
+// Device address of g_noalloc_x on `device`, which must be current.  Looked
+// up once per device; in host code the array's name is only a stand-in.
+static cudaError_t noalloc_scratch(int device, uint16_t** out) {
+    static std::mutex mu;
+    static uint16_t* addr[64] = {};
+    if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[device]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_x);
+        if (e != cudaSuccess) return e;
+        addr[device] = static_cast<uint16_t*>(p);
+    }
+    *out = addr[device];
+    return cudaSuccess;
+}
+
+cudaError_t launch_prefill_noalloc(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                                   const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
+                                   cudaStream_t s, const DeviceInfo& dev) {
+    if (static_cast<uint64_t>(M) * static_cast<uint64_t>(K) * sizeof(uint16_t) > Q4_NOALLOC_SCRATCH_BYTES)
+        return cudaErrorInvalidValue;  // rejected earlier by q4_gemm_noalloc
+    uint16_t* xh = nullptr;
+    const cudaError_t e = noalloc_scratch(dev.device, &xh);
+    if (e != cudaSuccess) return e;
+    return launch_prefill_tc(codes, scales, cb, x, xh, y, M, N, K, s, dev);
+}
+
 }  // namespace q4

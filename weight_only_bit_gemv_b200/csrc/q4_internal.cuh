@@ -50,6 +50,12 @@ cudaError_t launch_prefill(const uint8_t* codes, const uint16_t* scales, const u
                            const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
                            cudaStream_t s, const DeviceInfo& dev);
 
+// M > 16 with the x scratch in a fixed device array (q4_gemm_noalloc); the
+// caller has checked 2 * M * K <= Q4_NOALLOC_SCRATCH_BYTES.
+cudaError_t launch_prefill_noalloc(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                                   const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
+                                   cudaStream_t s, const DeviceInfo& dev);
+
 // Copy out and clear the timeout bits that a kernel family's bounded waits
 // set (synchronous; see q4_timeout_flags).
 cudaError_t take_gemv_tma_error(unsigned int* out);
