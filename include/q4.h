@@ -116,7 +116,15 @@ q4_status q4_dequant(const uint8_t* codes, const uint16_t* scales,
  * Each weight is rebuilt in registers as binary16 codebook[code]; products
  * with x are exact and accumulate in binary32; the group's scale multiplies
  * the group's binary32 partial sum.  The result matches the exact sum to
- * within 1e-4 * sum_k |W x| + 1e-6 per element.
+ * within 1e-4 * sum_k |W x| + 1e-6 per element.  Each element of y is
+ * written once by one thread block (no split of K across blocks), so the
+ * result does not depend on timing.
+ * Launch: with programmatic dependent launch.  The kernel may start while the
+ * preceding kernel on the stream is still running; before it waits for that
+ * kernel it only prefetches its inputs into L2 (which cannot return stale
+ * data), and it reads every input after the preceding kernel has completed.
+ * It also lets the next kernel start early; that kernel must itself wait
+ * before reading y (kernels launched without the attribute always do).
  * In: codes, scales, codebook, x [1][K] bf16.  Out: y [1][N] fp32.
  */
 q4_status q4_gemv(const uint8_t* codes, const uint16_t* scales,
@@ -191,12 +199,13 @@ int q4_last_cuda_error(void);
 int q4_abi_version(void);
 
 /*
- * q4_timeout_flags -- every wait inside the TMA and tensor-core kernels is
- * bounded (about two seconds); a wait that runs out sets a bit in a device
- * word, the kernel drains what it has in flight, frees its tensor memory and
- * exits, leaving its output incomplete.  This call synchronizes the current
- * device, stores the bits set since the last call in *flags (bits 0-15: the
- * M = 1 TMA GEMV; bits 16-31: the M > 16 tensor-core GEMM; 0 = no timeout)
+ * q4_timeout_flags -- every wait inside the bulk-copy and tensor-core
+ * kernels is bounded (about two seconds); a wait that runs out sets a bit in
+ * a device word, the kernel drains what it has in flight, frees its tensor
+ * memory and exits, leaving its output incomplete.  This call synchronizes the
+ * current device, stores the bits set since the last call in *flags (bits
+ * 0-15: the M = 1 GEMV, bit 8 there meaning that its shared-memory layout did
+ * not match the device; bits 16-31: the M > 16 tensor-core GEMM; 0 = none)
  * and clears them.  Not an operation of the method; a health check.
  * Returns Q4_ERR_NULL for a NULL flags, Q4_ERR_CUDA if a CUDA call fails.
  */

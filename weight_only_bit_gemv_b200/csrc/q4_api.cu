@@ -89,6 +89,8 @@ cudaError_t current_device_info(DeviceInfo* info) {
             (e = cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev)) ||
             (e = cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev)) ||
             (e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                                        dev)) ||
+            (e = cudaDeviceGetAttribute(&d.smem_reserved, cudaDevAttrReservedSharedMemoryPerBlock,
                                         dev)))
             return e;
         c.info[dev] = d;
@@ -211,7 +213,7 @@ q4_status q4_timeout_flags(uint32_t* flags) {
     if (!flags) return Q4_ERR_NULL;
     *flags = 0;
     unsigned int a = 0, b = 0;
-    cudaError_t e = take_gemv_tma_error(&a);
+    cudaError_t e = take_gemv_m1_error(&a);
     if (e == cudaSuccess) e = take_gemm_tc_error(&b);
     if (e != cudaSuccess) return cuda_fail(e);
     *flags = (a & 0xFFFFu) | ((b & 0xFFFFu) << 16);

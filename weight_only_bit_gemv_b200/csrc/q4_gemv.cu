@@ -291,7 +291,7 @@ cudaError_t launch_small_m(const uint8_t* codes, const uint16_t* scales, const u
                            const uint16_t* x, float* y, int M, int64_t N, int64_t K,
                            cudaStream_t s, const DeviceInfo& dev) {
     if (M == 1) {
-        cudaError_t e = launch_gemv_tma(codes, scales, cb, x, y, N, K, s, dev);
+        cudaError_t e = launch_gemv_m1(codes, scales, cb, x, y, N, K, s, dev);
         if (e != cudaErrorNotSupported) return e;
         (void)cudaGetLastError();
     }

@@ -1,0 +1,611 @@
+// q4_gemv_m1.cu -- the M = 1 decode GEMV on sm_100a.
+//
+// What it computes: y[n] = sum_g scale[n][g] * sum_{k in g} cb[code(n,k)] * x[k]
+// ("deep-fold", "Method": 64-weight groups, four-bit codes, one FP16 scale;
+// the decode GEMV rebuilds values while it multiplies and writes no dense
+// matrix; "Trapetum" overview, "The bandwidth law": decode time is the time
+// to read the weight bytes).
+//
+// Why this shape.  Decode streams 0.53125 bytes per weight, so the kernel is
+// an HBM stream with the decode hidden under it.
+//  * DRAM sees long contiguous reads issued as few, large bulk copies.  CTA c
+//    owns the rows [N c / grid, N (c + 1) / grid), a contiguous range of the
+//    code matrix.  A producer warp copies it into a shared-memory ring with
+//    1-D bulk copies (cp.async.bulk), one 16-row tile (or a 16-row x 2 KB
+//    slice of it) per stage: a whole tile of rows up to 2 KB long is one
+//    contiguous copy, longer rows are copied one ~2 KB row segment at a
+//    time.  On B200 a bulk copy costs about 50 ns of its SM's copy engine
+//    whatever its size, so copies of 1 KB or less cap the stream far below
+//    the HBM rate, and reads of 64-128 bytes of many rows at a time (per-lane
+//    loads, 2-D tensor boxes) lose DRAM efficiency; the layout above avoids
+//    both.
+//  * Each code byte indexes a 256-entry byte -> half2 table (cb[lo nibble],
+//    cb[hi nibble]) held once per lane (entry b of lane l at 256 b + 4 l, at
+//    the start of dynamic shared memory), so one PRMT of (code word, 4 l)
+//    forms the address, the table's shared-window base is an immediate of
+//    the load, and the 32 lanes hit 32 banks; one LDS returns two weights.
+//  * The weights are the A operand of mma.sync m16n8k16 (binary16 products
+//    are exact, sums are fp32).  A warp's unit is 16 rows x 256 k (two spans
+//    of 128 k, four groups).  In pass A the even rows of the tile take span
+//    2u and the odd rows span 2u + 1; in pass B they swap.  Lane (g, tq) reads
+//    16 code bytes of rows g and g + 8, so a quarter warp (rows g, g + 1)
+//    always reads 128 distinct bytes (no bank conflicts, no padding).  The B
+//    operand's columns 0-3 hold x of the unit's four groups, each zero
+//    outside its group, so one chain of eight MMAs per pass yields every
+//    row's per-group sums in columns 0-3; lane tq in {0, 1} keeps span
+//    2u + tq of its rows and scales each group's fp32 sum by its own scale.
+//  * x is rounded to binary16 once per CTA into shared memory in that
+//    column layout (for K <= 8192 inside the unused half of the table rows).
+//    Scales are read from global memory by the consumers, stages ahead.
+//  * The warps of a CTA add their tile sums into a shared-memory row
+//    accumulator; the CTA writes each y element once (no split-K between
+//    CTAs, no zeroing of y, no global atomics).
+//  * Programmatic dependent launch: the kernel lets the next kernel on the
+//    stream launch at once, prefetches the first stages of its weights into
+//    L2 (a prefetch only warms the cache, so it never reads stale data), and
+//    waits for the preceding kernel before it reads any input.
+#include "q4_internal.cuh"
+#include "q4_sm100.cuh"
+
+namespace q4 {
+
+__device__ unsigned int g_gemv_m1_error;
+
+namespace {
+
+constexpr int kCW = 8;                    // consumer warps
+constexpr int kUPW = 2;                   // units per consumer warp per stage
+constexpr int kThreads = (kCW + 1) * 32;  // + one producer warp
+constexpr int kBase = 1024;               // shared-window address of dynamic shared memory
+constexpr int kLutBytes = 65536;          // 256 rows of 256 bytes; lane copies in the first 128
+constexpr int kSpan = 128;                // k per span (64 code bytes)
+constexpr int kMaxKC = 2048;              // code bytes of a row per stage
+constexpr int kPassTiles = 128;           // tiles per pass of the shared row accumulator
+constexpr int kAhead = 3;                 // scale prefetch distance, in stages
+constexpr int kMaxStages = 6;
+constexpr int kXEmbedSpans = 64;          // spans whose x fits in the table rows' free halves
+constexpr int kXRounds = 13;              // x chunk loads per consumer thread: K <= 13 * 256 * 8
+constexpr uint32_t kAccOff = kLutBytes;
+constexpr uint32_t kBarOff = kAccOff + kPassTiles * 16 * 4;
+constexpr uint32_t kXOff = kBarOff + 128;
+
+struct M1 {
+    const uint8_t* codes;
+    const uint16_t* scales;
+    const uint16_t* cb;
+    const uint16_t* x;
+    float* y;
+    int N, K, G, S;  // S = spans of 128 k (the last may hold one group)
+    int SP;          // S rounded up to even: x holds a zero span S when S is odd
+    int rowbytes;    // K / 2
+    int KC;          // code bytes of a row per stage (the ring's row pitch)
+    int C;           // stages per 16-row tile
+    int NS;          // ring stages
+    uint32_t ring_off, stage_bytes;
+};
+
+// Scale reads go through L1: the 8 consumer warps read neighbouring pairs of
+// the same rows, so most of them hit lines another warp brought in (measured:
+// non-allocating scale loads cost a quarter of the kernel's throughput).
+__device__ __forceinline__ uint32_t ldg_u32(const void* p) {
+    uint32_t v;
+    asm("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ldg_u16(const void* p) {
+    unsigned short v;
+    asm("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
+// Table read: `off` is a dynamic-shared-memory offset.
+__device__ __forceinline__ uint32_t lds32_dyn(uint32_t off) {
+    uint32_t v;
+    asm("ld.shared.b32 %0, [%1 + %2];" : "=r"(v) : "r"(off), "n"(kBase));
+    return v;
+}
+
+template <int kOff>
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4 + %5];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "r"(addr), "n"(kOff));
+    return v;
+}
+
+// Ring reads stay behind the mbarrier wait that precedes them (volatile).
+template <int kOff>
+__device__ __forceinline__ uint4 lds128_ring(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4 + %5];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr), "n"(kOff));
+    return v;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// The scales of rows [row0, row1) lie contiguously; warm L2 with them (the
+// range is shrunk to whole 16-byte blocks inside the buffer).
+__device__ __forceinline__ void prefetch_scales_l2(const uint16_t* scales, int64_t G, int64_t N,
+                                                   int row0, int row1) {
+    const uint64_t b0 = (static_cast<uint64_t>(row0) * G * 2 + 15) & ~15ull;
+    const uint64_t b1 = (static_cast<uint64_t>(row1) * G * 2) & ~15ull;
+    const uint64_t end = (static_cast<uint64_t>(N) * G * 2) & ~15ull;
+    const uint64_t e = b1 < end ? b1 : end;
+    if (e > b0)
+        prefetch_l2(reinterpret_cast<const uint8_t*>(scales) + b0, static_cast<uint32_t>(e - b0));
+}
+
+__device__ __forceinline__ uint32_t cvt_bf16x2_f16x2(uint32_t w) {
+    const __half2 h = __floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float f16_lo(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu)));
+}
+__device__ __forceinline__ float f16_hi(uint32_t w) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
+}
+
+// Table entry (cb[lo], cb[hi]) of byte kByte of `word` for this lane: offset
+// [lane*4, code byte, 0, 0] from the start of dynamic shared memory.
+template <int kByte>
+__device__ __forceinline__ uint32_t lut(uint32_t word, uint32_t lane4) {
+    return lds32_dyn(__byte_perm(word, lane4, 0x5504 | (kByte << 4)));
+}
+
+__device__ __forceinline__ uint32_t lane4_of(int lane) { return static_cast<uint32_t>(lane) * 4u; }
+
+// One pass over the 128 k of this lane's row slots: eight MMAs in two
+// independent chains of four (the sums of k-steps 0-3 and 4-7), so that a
+// warp keeps more MMAs in flight.
+__device__ __forceinline__ void pass_mma(uint4 lo, uint4 hi, const uint32_t (&xr)[16],
+                                         uint32_t lane4, float (&d)[4], float (&e)[4]) {
+    const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w};
+    const uint32_t wh[4] = {hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        const uint32_t l = wl[t >> 1], h = wh[t >> 1];
+        uint32_t a[4];
+        if (t & 1) {
+            a[0] = lut<2>(l, lane4);
+            a[1] = lut<2>(h, lane4);
+            a[2] = lut<3>(l, lane4);
+            a[3] = lut<3>(h, lane4);
+        } else {
+            a[0] = lut<0>(l, lane4);
+            a[1] = lut<0>(h, lane4);
+            a[2] = lut<1>(l, lane4);
+            a[3] = lut<1>(h, lane4);
+        }
+        if (t < 4)
+            mma_16816(d, a, xr[2 * t], xr[2 * t + 1], d);
+        else
+            mma_16816(e, a, xr[2 * t], xr[2 * t + 1], e);
+    }
+}
+
+// Scales of groups 2s, 2s + 1 of a row (`srow` = its first scale) as a
+// binary16 pair; the second repeats the first when 2s + 1 == G (it then
+// multiplies a zero sum).
+template <bool kEvenG>
+__device__ __forceinline__ uint32_t load_scales(const M1& p, const uint16_t* srow, int s) {
+    const uint16_t* q = srow + 2 * s;
+    if (kEvenG) return ldg_u32(q);
+    return ldg_u16(q) | (ldg_u16(q + (2 * s + 1 < p.G ? 1 : 0)) << 16);
+}
+
+template <bool kEvenG, bool kWhole, bool kXEmb>
+__global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, tq = lane & 3;
+
+    // The next kernel on the stream may launch now; it waits for this one
+    // before it reads anything this one writes.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    // Table reads use the dynamic-shared-memory base as an immediate; a
+    // different base is reported (bit 8 of q4_timeout_flags) instead of used.
+    const uint32_t base = smem_u32(smem);
+    if (base != static_cast<uint32_t>(kBase)) {
+        if (tid == 0) atomicOr(&g_gemv_m1_error, 0x100u);
+        return;
+    }
+    const uint32_t bars = base + kBarOff;
+    const int NS = p.NS;
+    const int r0 = static_cast<int>(static_cast<int64_t>(p.N) * blockIdx.x / gridDim.x);
+    const int r1 = static_cast<int>(static_cast<int64_t>(p.N) * (blockIdx.x + 1) / gridDim.x);
+    const int nrows = r1 - r0;
+    const int T = (nrows + 15) >> 4;
+    const int total = T * p.C;  // stages of this CTA
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bars + 8u * s, 1);           // full: the producer's expect_tx
+            mbar_init(bars + 8u * (NS + s), kCW);  // empty: one arrival per consumer warp
+        }
+        fence_mbar_init();
+    }
+    // Warm L2 with the first stage while the preceding kernel finishes (more
+    // would queue ahead of the set-up's reads of x in DRAM).
+    if (warp == kCW) {
+        for (int i = 0; i < 1 && i < total; ++i) {
+            const int t = i / p.C, c = i - t * p.C;
+            const int rows = min(16, nrows - 16 * t);
+            if (kWhole) {
+                if (lane == 0)
+                    prefetch_l2(p.codes + static_cast<int64_t>(r0 + 16 * t) * p.rowbytes,
+                                static_cast<uint32_t>(rows * p.rowbytes));
+            } else if (lane < rows) {
+                prefetch_l2(p.codes + static_cast<int64_t>(r0 + 16 * t + lane) * p.rowbytes + c * p.KC,
+                            static_cast<uint32_t>(min(p.KC, p.rowbytes - c * p.KC)));
+            }
+        }
+    }
+    if (warp == kCW && lane == 31)
+        prefetch_scales_l2(p.scales, p.G, p.N, r0, r0 + min(nrows, 32));
+    // x and the codebook too: a prefetch is coherent (L2 is the point of
+    // coherence), so this is safe even if the preceding kernel writes them;
+    // the reads below, after the wait, then find them in L2.
+    if (warp == kCW && lane == 30) prefetch_l2(p.x, static_cast<uint32_t>(p.K) * 2u);
+    if (warp == kCW && lane == 29) prefetch_l2(p.cb, 32u);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __syncthreads();
+
+    if (warp == kCW) {
+        // ------------------------------ producer ------------------------------
+        // The set-up's reads of x and the codebook go out first; the weight
+        // stream starts once every consumer has issued them.
+        asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
+        const uint32_t ring = base + p.ring_off;
+        int slot = 0, t = 0, c = 0;
+        uint32_t eparity = 1;  // parity of the empty phase to wait for (round - 1)
+        for (int i = 0; i < total; ++i) {
+            if (i >= NS) {
+                uint32_t ok = 1;
+                if (lane == 0) ok = mbar_wait(bars + 8u * (NS + slot), eparity) ? 1u : 0u;
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) {
+                    if (lane == 0) atomicOr(&g_gemv_m1_error, 0x200u);
+                    break;
+                }
+            }
+            const int rows = min(16, nrows - 16 * t);
+            const uint32_t dst = ring + slot * p.stage_bytes;
+            const uint32_t full = bars + 8u * slot;
+            // The consumers read scales with small loads; have the tile two
+            // ahead's scales in L2 by then (one contiguous block per tile).
+            if (c == 0 && lane == 31 && 16 * (t + 2) < nrows)
+                prefetch_scales_l2(p.scales, p.G, p.N, r0 + 16 * (t + 2),
+                                   r0 + min(nrows, 16 * (t + 3)));
+            if (kWhole) {
+                if (lane == 0) {
+                    const uint32_t bytes = static_cast<uint32_t>(rows * p.rowbytes);
+                    mbar_arrive_expect_tx(full, bytes);
+                    bulk_load(dst, p.codes + static_cast<int64_t>(r0 + 16 * t) * p.rowbytes, bytes,
+                              full);
+                }
+            } else {
+                const uint32_t bytes = static_cast<uint32_t>(min(p.KC, p.rowbytes - c * p.KC));
+                if (lane == 0) mbar_arrive_expect_tx(full, bytes * rows);
+                __syncwarp();
+                if (lane < rows)
+                    bulk_load(dst + lane * p.KC,
+                              p.codes + static_cast<int64_t>(r0 + 16 * t + lane) * p.rowbytes +
+                                  c * p.KC,
+                              bytes, full);
+            }
+            if (++c == p.C) {
+                c = 0;
+                ++t;
+            }
+            if (++slot == NS) {
+                slot = 0;
+                eparity ^= 1u;
+            }
+        }
+        // Leave only once this warp's copies have landed (bounded).
+        if (lane == 0) {
+            for (int i = (total > NS ? total - NS : 0); i < total; ++i)
+                if (!mbar_wait(bars + 8u * (i % NS), (i / NS) & 1)) {
+                    atomicOr(&g_gemv_m1_error, 0x400u);
+                    break;
+                }
+        }
+        return;
+    }
+
+    // ------------------------------- consumers ------------------------------
+    float* acc_s = reinterpret_cast<float*>(smem + kAccOff);
+    {
+        // Issue every global read of the set-up at once (the codebook and all
+        // of x: one 16-byte chunk per thread and round), then build the table
+        // and the x layout: one memory latency instead of one per round.
+        const uint32_t cbv = p.cb[lane & 15];
+        const int nx = p.K >> 3;  // 16-byte chunks of x (8 values)
+        uint4 xv[kXRounds];
+#pragma unroll
+        for (int i = 0; i < kXRounds; ++i) {
+            const int r = tid + i * kCW * 32;
+            xv[i] = r < nx ? __ldg(reinterpret_cast<const uint4*>(p.x) + r) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
+        // byte -> (cb[lo], cb[hi]) table, one copy per lane
+        for (int b = warp; b < 256; b += kCW) {
+            const uint32_t lo = __shfl_sync(0xFFFFFFFFu, cbv, b & 15);
+            const uint32_t hi = __shfl_sync(0xFFFFFFFFu, cbv, b >> 4);
+            *reinterpret_cast<uint32_t*>(smem + b * 256 + lane * 4) = lo | (hi << 16);
+        }
+        // x as binary16: 16-byte chunk (span s, quarter q, parity par, j)
+        // holds x[128 s + 32 j + 8 q, +8) when par == j / 2 (the column of
+        // that group), else zeros; chunks past K are zeros.
+        auto chunk_off = [&](int s, int q, int par, int j) -> uint32_t {
+            return kXEmb ? (4 * s + q) * 256 + 128 + par * 64 + j * 16
+                         : kXOff + s * 512 + q * 128 + par * 64 + j * 16;
+        };
+#pragma unroll
+        for (int i = 0; i < kXRounds; ++i) {
+            const int r = tid + i * kCW * 32;
+            if (r < nx) {
+                const int k = 8 * r;
+                const int s = k >> 7, j = (k >> 5) & 3, q = (k >> 3) & 3;
+                uint4 h;
+                h.x = cvt_bf16x2_f16x2(xv[i].x);
+                h.y = cvt_bf16x2_f16x2(xv[i].y);
+                h.z = cvt_bf16x2_f16x2(xv[i].z);
+                h.w = cvt_bf16x2_f16x2(xv[i].w);
+                *reinterpret_cast<uint4*>(smem + chunk_off(s, q, j >> 1, j)) = h;
+                *reinterpret_cast<uint4*>(smem + chunk_off(s, q, 1 - (j >> 1), j)) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        // the spans that reach past K: their chunks beyond K are zeros
+        for (int c = (p.S - 1) * 32 + tid; c < p.SP * 32; c += kCW * 32) {
+            const int j = c & 3, par = (c >> 2) & 1, q = (c >> 3) & 3, s = c >> 5;
+            if (s * kSpan + 32 * j + 8 * q >= p.K)
+                *reinterpret_cast<uint4*>(smem + chunk_off(s, q, par, j)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+    constexpr uint32_t kXSpan = kXEmb ? 1024u : 512u;  // x bytes between spans
+    const int upk = p.KC >> 7;                         // units (256 k) per full stage
+    // this lane's code offsets in a stage: rows g and g + 8, pass A and B
+    const uint32_t ring_lane = base + p.ring_off + g * p.KC + 16 * tq;
+    const uint32_t offA = 64 * (g & 1), offB = 64 - offA;
+    const uint32_t rowhi = 8 * p.KC;
+    const bool use_a = (tq & 1) == (g & 1);
+    bool bad = false;
+
+    // Scales of the stages ahead ([0] = the current stage's): for unit j of
+    // this warp, span 2U + (tq & 1) of rows g and g + 8.  The prefetch cursor
+    // (st, sc) runs kAhead stages ahead of the consumer's.
+    uint32_t sc[kAhead][kUPW][2];
+    int st = 0, scc = 0, sleft = total;
+    const uint16_t* srow_lo = nullptr;
+    const uint16_t* srow_hi = nullptr;
+    auto scale_rows = [&]() {
+        srow_lo = p.scales + static_cast<int64_t>(r0 + min(16 * st + g, nrows - 1)) * p.G;
+        srow_hi = p.scales + static_cast<int64_t>(r0 + min(16 * st + g + 8, nrows - 1)) * p.G;
+    };
+    auto next_scales = [&](uint32_t (&out)[kUPW][2]) {
+#pragma unroll
+        for (int j = 0; j < kUPW; ++j) out[j][0] = out[j][1] = 0u;
+        if (sleft > 0) {
+#pragma unroll
+            for (int j = 0; j < kUPW; ++j) {
+                const int sp = min(2 * (scc * upk + warp + kCW * j) + (tq & 1), p.S - 1);
+                out[j][0] = load_scales<kEvenG>(p, srow_lo, sp);
+                out[j][1] = load_scales<kEvenG>(p, srow_hi, sp);
+            }
+            --sleft;
+            if (++scc == p.C) {
+                scc = 0;
+                ++st;
+                scale_rows();
+            }
+        }
+    };
+    scale_rows();
+#pragma unroll
+    for (int i = 0; i < kAhead; ++i) next_scales(sc[i]);
+
+    // One unit: two passes of eight MMAs; lane tq in {0, 1} adds span
+    // 2U + tq of rows g and g + 8, each group scaled by its own scale.
+    auto unit = [&](uint32_t a, const uint32_t (&xr)[16], const uint32_t (&s)[2], float& acc_lo,
+                    float& acc_hi) {
+        const uint4 loA = lds128_ring<0>(a + offA), hiA = lds128_ring<0>(a + offA + rowhi);
+        const uint4 loB = lds128_ring<0>(a + offB), hiB = lds128_ring<0>(a + offB + rowhi);
+        float dA[4] = {0.f, 0.f, 0.f, 0.f}, eA[4] = {0.f, 0.f, 0.f, 0.f};
+        float dB[4] = {0.f, 0.f, 0.f, 0.f}, eB[4] = {0.f, 0.f, 0.f, 0.f};
+        pass_mma(loA, hiA, xr, lane4_of(lane), dA, eA);
+        pass_mma(loB, hiB, xr, lane4_of(lane), dB, eB);
+        const float d0 = use_a ? dA[0] + eA[0] : dB[0] + eB[0];
+        const float d1 = use_a ? dA[1] + eA[1] : dB[1] + eB[1];
+        const float d2 = use_a ? dA[2] + eA[2] : dB[2] + eB[2];
+        const float d3 = use_a ? dA[3] + eA[3] : dB[3] + eB[3];
+        acc_lo = fmaf(f16_lo(s[0]), d0, acc_lo);
+        acc_lo = fmaf(f16_hi(s[0]), d1, acc_lo);
+        acc_hi = fmaf(f16_lo(s[1]), d2, acc_hi);
+        acc_hi = fmaf(f16_hi(s[1]), d3, acc_hi);
+    };
+    auto load_x = [&](uint32_t xa, uint32_t (&xr)[16]) {
+        uint4 x0, x1, x2, x3;
+        if (kXEmb) {
+            x0 = lds128<0>(xa);
+            x1 = lds128<256>(xa);
+            x2 = lds128<512>(xa);
+            x3 = lds128<768>(xa);
+        } else {
+            x0 = lds128<0>(xa);
+            x1 = lds128<128>(xa);
+            x2 = lds128<256>(xa);
+            x3 = lds128<384>(xa);
+        }
+        const uint32_t v[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
+                                x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xr[i] = v[i];
+    };
+
+    bool started = false;
+    uint32_t xlane = 0;
+    uint32_t xw[kUPW][16];  // whole rows: this warp's units never change, nor their x
+    int slot = 0;
+    uint32_t fparity = 0;
+    for (int pt0 = 0; pt0 < T; pt0 += kPassTiles) {
+        const int pt1 = min(T, pt0 + kPassTiles);
+        for (int i = tid; i < kPassTiles * 16; i += kCW * 32) acc_s[i] = 0.f;
+        asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+        if (!started) {
+            // formed after the first consumer barrier: the empty asm keeps every
+            // x read below it
+            xlane = base + (kXEmb ? 128u : kXOff) + ((g >> 1) & 1) * kXSpan + (g & 1) * 64 + tq * 16;
+            asm volatile("" : "+r"(xlane)::"memory");
+            if (kWhole) {
+#pragma unroll
+                for (int j = 0; j < kUPW; ++j)
+                    load_x(xlane + static_cast<uint32_t>(warp + kCW * j) * (2 * kXSpan), xw[j]);
+            }
+            started = true;
+        }
+        for (int t = pt0; t < pt1; ++t) {
+            float acc_lo = 0.f, acc_hi = 0.f;
+            for (int c = 0; c < p.C; ++c) {
+                if (!bad && !mbar_wait(bars + 8u * slot, fparity)) {
+                    bad = true;
+                    if (lane == 0) atomicOr(&g_gemv_m1_error, 0x800u);
+                }
+                const int units = (min(p.KC, p.rowbytes - c * p.KC) + 127) >> 7;
+                const uint32_t a0 = ring_lane + slot * p.stage_bytes + 128 * warp;
+#pragma unroll
+                for (int j = 0; j < kUPW; ++j) {
+                    if (!bad && warp + kCW * j < units) {
+                        if (kWhole) {
+                            unit(a0 + 128 * kCW * j, xw[j], sc[0][j], acc_lo, acc_hi);
+                        } else {
+                            uint32_t xr[16];
+                            load_x(xlane + static_cast<uint32_t>(c * upk + warp + kCW * j) * (2 * kXSpan),
+                                   xr);
+                            unit(a0 + 128 * kCW * j, xr, sc[0][j], acc_lo, acc_hi);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + 8u * (NS + slot));
+                if (++slot == NS) {
+                    slot = 0;
+                    fparity ^= 1u;
+                }
+#pragma unroll
+                for (int i = 0; i < kAhead - 1; ++i)
+#pragma unroll
+                    for (int j = 0; j < kUPW; ++j) {
+                        sc[i][j][0] = sc[i + 1][j][0];
+                        sc[i][j][1] = sc[i + 1][j][1];
+                    }
+                next_scales(sc[kAhead - 1]);
+            }
+            // lanes tq = 0, 1 hold the two spans' sums of rows g, g + 8
+            acc_lo += __shfl_xor_sync(0xFFFFFFFFu, acc_lo, 1);
+            acc_hi += __shfl_xor_sync(0xFFFFFFFFu, acc_hi, 1);
+            if (tq == 0) {
+                const int rl = 16 * (t - pt0) + g;
+                if (16 * t + g < nrows) atomicAdd(acc_s + rl, acc_lo);
+                if (16 * t + g + 8 < nrows) atomicAdd(acc_s + rl + 8, acc_hi);
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+        const int row_end = min(nrows, 16 * pt1);
+        for (int r = 16 * pt0 + tid; r < row_end; r += kCW * 32) p.y[r0 + r] = acc_s[r - 16 * pt0];
+        asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+    }
+}
+
+template <bool kEvenG, bool kWhole, bool kXEmb>
+cudaError_t launch_variant(const M1& p, int grid, int smem, int slot, cudaStream_t s,
+                           const DeviceInfo& dev) {
+    auto kern = gemv_m1_kernel<kEvenG, kWhole, kXEmb>;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem, slot, dev.device);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+}  // namespace
+
+cudaError_t take_gemv_m1_error(unsigned int* out) {
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_gemv_m1_error, sizeof(unsigned int));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_gemv_m1_error, &zero, sizeof(unsigned int));
+    return e;
+}
+
+cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                           const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
+                           const DeviceInfo& dev) {
+    if (dev.smem_reserved != kBase) return cudaErrorNotSupported;
+    M1 p{};
+    p.codes = codes;
+    p.scales = scales;
+    p.cb = cb;
+    p.x = x;
+    p.y = y;
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.G = static_cast<int>(K / kGroup);
+    p.S = (p.K + kSpan - 1) / kSpan;
+    p.SP = p.S + (p.S & 1);
+    p.rowbytes = p.K / 2;
+    // A stage is 16 rows x KC bytes.  Rows up to 2 KB whose length is a
+    // multiple of 128 bytes travel whole (a tile is one contiguous copy);
+    // longer rows in C segments of KC bytes (a multiple of 128).
+    const bool whole = p.rowbytes <= kMaxKC && p.rowbytes % 128 == 0;
+    if (whole) {
+        p.C = 1;
+        p.KC = p.rowbytes;
+    } else {
+        p.C = (p.rowbytes + kMaxKC - 1) / kMaxKC;
+        p.KC = ((p.rowbytes + p.C - 1) / p.C + 127) / 128 * 128;
+    }
+    if (p.K > kXRounds * kCW * 32 * 8) return cudaErrorNotSupported;
+    const bool xemb = p.SP <= kXEmbedSpans;
+    const uint32_t x_end = xemb ? kXOff : kXOff + static_cast<uint32_t>(p.SP) * 512u;
+    p.ring_off = (x_end + 127u) & ~127u;
+    p.stage_bytes = static_cast<uint32_t>(16 * p.KC);
+    const int room = dev.smem_optin - static_cast<int>(p.ring_off) - 128;  // 128: read slack
+    int ns = room / static_cast<int>(p.stage_bytes);
+    if (ns > kMaxStages) ns = kMaxStages;
+    if (ns < 2) return cudaErrorNotSupported;
+    p.NS = ns;
+    const int smem = static_cast<int>(p.ring_off + ns * p.stage_bytes) + 128;
+
+    const int64_t tiles = (N + 15) / 16;
+    const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+    const bool even = (p.G & 1) == 0;
+    if (whole) {
+        return even ? launch_variant<true, true, true>(p, grid, smem, 16, s, dev)
+                    : launch_variant<false, true, true>(p, grid, smem, 17, s, dev);
+    }
+    if (xemb)
+        return even ? launch_variant<true, false, true>(p, grid, smem, 18, s, dev)
+                    : launch_variant<false, false, true>(p, grid, smem, 19, s, dev);
+    return even ? launch_variant<true, false, false>(p, grid, smem, 20, s, dev)
+                : launch_variant<false, false, false>(p, grid, smem, 21, s, dev);
+}
+
+}  // namespace q4

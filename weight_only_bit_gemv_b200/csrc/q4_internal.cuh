@@ -20,6 +20,7 @@ struct DeviceInfo {
     int sm_count;
     int cc_major, cc_minor;
     int smem_optin;  // max dynamic shared memory per block (opt-in)
+    int smem_reserved;  // shared memory the system reserves per block (ahead of user shared memory)
 };
 // Fills *info for the current device; returns cudaSuccess or the failing code.
 cudaError_t current_device_info(DeviceInfo* info);
@@ -40,11 +41,12 @@ cudaError_t launch_dequant(const uint8_t* codes, const uint16_t* scales, const u
 cudaError_t launch_small_m(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int M, int64_t N, int64_t K,
                            cudaStream_t s, const DeviceInfo& dev);
-// M = 1: TMA-fed, warp-specialized decode GEMV.  Returns cudaErrorNotSupported
-// when the shape does not fit it (shared-memory budget).
-cudaError_t launch_gemv_tma(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
-                            const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
-                            const DeviceInfo& dev);
+// M = 1: bulk-copy-fed decode GEMV, one row range per CTA, launched with
+// programmatic dependent launch.  Returns cudaErrorNotSupported when the
+// shape does not fit it (K too large for its shared-memory layout).
+cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                           const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
+                           const DeviceInfo& dev);
 // M > 16: tcgen05 tensor-core GEMM with TMEM accumulators.
 cudaError_t launch_prefill(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
@@ -58,7 +60,7 @@ cudaError_t launch_prefill_noalloc(const uint8_t* codes, const uint16_t* scales,
 
 // Copy out and clear the timeout bits that a kernel family's bounded waits
 // set (synchronous; see q4_timeout_flags).
-cudaError_t take_gemv_tma_error(unsigned int* out);
+cudaError_t take_gemv_m1_error(unsigned int* out);
 cudaError_t take_gemm_tc_error(unsigned int* out);
 
 // ---------------------------------------------------------------------------
