@@ -53,6 +53,27 @@ def peaks():
         return 6650.0, 1590.0, "fallback"
 
 
+# DRAM bytes (read + write) of one q4_gemv launch on the gate_up linear
+# (4096 -> 22016) from an ncu capture, with the SHA-1 of the kernel source it
+# was taken on; when the source changes the figure no longer applies and the
+# bench reports null.
+GEMV_TRAFFIC = {"bytes": 47957248 + 1536,
+                "source_sha1": "b1a19fc116b11bd24b9578842bf1f7edb4419cb1",
+                "capture": "ncu --set full --clock-control none -k regex:gemv_m1 -s 2 -c 1 "
+                           "python -m weight_only_bit_gemv_b200.profile_case --M 1 --iters 5 "
+                           "--copies 2 --workload llama2_7b_layer --linear gate_up"}
+
+
+def gemv_traffic():
+    import hashlib
+    path = os.path.join(ROOT, "weight_only_bit_gemv_b200", "csrc", "q4_gemv_m1.cu")
+    try:
+        sha = hashlib.sha1(open(path, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return GEMV_TRAFFIC["bytes"] if sha == GEMV_TRAFFIC["source_sha1"] else None
+
+
 def algo_bytes(M, N, K):
     """Algorithmic bytes of one q4 matmul: codes + scales + x + y + codebook."""
     return N * K // 2 + N * (K // GROUP) * 2 + M * K * 2 + M * N * 4 + 32
@@ -202,11 +223,19 @@ def run_ours(args, world, rank, local):
     stream.synchronize()
     graphs, _ = capture_graphs(lins, cb, stream, with_events=False)
     egraphs, eevents = capture_graphs(lins, cb, stream, with_events=True)
+    # One graph of COPIES consecutive steps (one per weight copy): a replay
+    # submits 4 * COPIES launches, so host submission never paces the GPU.
+    g_multi = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_multi, stream=stream):
+        for c in range(COPIES):
+            for L in lins:
+                q4.q4_gemv(L["copies"][c][0], L["copies"][c][1], cb, L["x"], L["y"])
 
     K, W = args.steps, args.warmup
     with torch.cuda.stream(stream):
         for i in range(W):
             graphs[i % COPIES].replay()
+        g_multi.replay()
     stream.synchronize()
 
     # ---- timed region: exactly K steps -------------------------------------
@@ -218,8 +247,10 @@ def run_ours(args, world, rank, local):
     t1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         t0.record()
-        for i in range(K):
-            graphs[i % COPIES].replay()
+        for i in range(K // COPIES):
+            g_multi.replay()
+        for i in range(K % COPIES):
+            graphs[i].replay()
         t1.record()
     t1.synchronize()
     barrier(world)
@@ -243,7 +274,27 @@ def run_ours(args, world, rank, local):
     per_ms = [statistics.mean(p) for p in per]
     dom = max(range(len(lins)), key=lambda j: algo_bytes(1, lins[j]["lin"].N, lins[j]["lin"].K))
     dom_bytes = algo_bytes(1, lins[dom]["lin"].N, lins[dom]["lin"].K)
-    dom_gbs = dom_bytes / (per_ms[dom] * 1e-3) / 1e9
+    # The dominant kernel timed on its own: one graph of COPIES back-to-back
+    # launches over the rotating weight copies (events around the graph; an
+    # event between launches would also time the launch gap it creates).
+    Ld = lins[dom]
+    g_dom = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_dom, stream=stream):
+        for c in range(COPIES):
+            q4.q4_gemv(Ld["copies"][c][0], Ld["copies"][c][1], cb, Ld["x"], Ld["y"])
+    reps_dom = max(4, min(K, 200))
+    d0 = torch.cuda.Event(enable_timing=True)
+    d1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g_dom.replay()
+        d0.record()
+        for _ in range(reps_dom):
+            g_dom.replay()
+        d1.record()
+    d1.synchronize()
+    dom_ms = d0.elapsed_time(d1) / (reps_dom * COPIES)
+    dom_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
 
     # ---- end to end through the Python API with host buffers -----------------
     xh = [torch.empty((1, L["lin"].K), dtype=torch.bfloat16).pin_memory() for L in lins]
@@ -319,7 +370,10 @@ def run_ours(args, world, rank, local):
             "peak_source": peak_src,
             "unit": "GB/s",
             "frac": round(dom_gbs / hbm_peak, 4),
-            "traffic": None,
+            "traffic": gemv_traffic(),
+            "algorithmic_bytes": dom_bytes,
+            "us_per_launch": round(dom_ms * 1e3, 3),
+            "timing": f"{COPIES} back-to-back launches in one CUDA graph over rotating weight copies",
         },
         "e2e": {
             "value": round(world * bytes_step / (e2e_ms * 1e-3) / 1e9, 2),
@@ -354,10 +408,10 @@ def bench_prefill(dev, cb, stream, tc_peak, M=256):
         x = synth.activations_device(synth.x_seed(seed) + M, M, lin.K, dev)
         y = torch.empty((M, lin.N), dtype=torch.float32, device=dev)
         with torch.cuda.stream(stream):
-            for _ in range(3):
+            for _ in range(10):
                 q4.q4_gemm(codes, scales, cb, x, y)
             stream.synchronize()
-            reps = 10
+            reps = 20
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record()
