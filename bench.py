@@ -332,6 +332,10 @@ def run_ours(args, world, rank, local):
     if not args.no_gemm:
         gemm = bench_prefill(dev, cb, stream, tc_peak, M=256)
 
+    # ---- other workloads: a full 8B decode step, small-M verify batches --------
+    step8b = None if args.no_step else bench_decode_step(dev, cb, stream, hbm_peak)
+    smallm = None if args.no_smallm else bench_small_m(dev, cb, stream, hbm_peak)
+
     # ---- CPU baseline: the oracle on the host --------------------------------
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -388,6 +392,10 @@ def run_ours(args, world, rank, local):
     }
     if gemm is not None:
         line["gemm_prefill"] = gemm
+    if step8b is not None:
+        line["decode_step_llama31_8b"] = step8b
+    if smallm is not None:
+        line["small_m_verify"] = smallm
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if rank == 0:
@@ -442,6 +450,106 @@ def bench_prefill(dev, cb, stream, tc_peak, M=256):
             "timing": "CUDA graph of 4 back-to-back q4_gemm calls (x conversion, y zeroing when K "
                       "is split, and the tensor-core GEMM), replayed 5 times",
             "note": "no L2 flush: each linear is 37-253 MB of packed weights, read once per launch"}
+
+
+def bench_decode_step(dev, cb, stream, hbm_peak, reps=20):
+    """Llama-3.1-8B decode step at M = 1: 32 layers x (qkv, o, gate_up, down) +
+    lm_head, one q4_gemv per linear (129 launches) in one CUDA graph, every
+    layer with its own seeded weights (3.99 GB packed, resident in HBM)."""
+    import torch
+    import weight_only_bit_gemv_b200 as q4
+    wl = synth.WORKLOADS["llama31_8b_step"]
+    layers = [lin for lin in wl.linears if lin.name != "lm_head"]
+    head = [lin for lin in wl.linears if lin.name == "lm_head"][0]
+    order = [(layer, lin) for layer in range(32) for lin in layers] + [(0, head)]
+    packs, xs, ys = [], {}, []
+    for layer, lin in order:
+        seed = synth.seed_for(wl.index, layer, lin.name)
+        w = synth.weights_device(seed, lin.N, lin.K, wl.w_std, dev)
+        codes, scales = q4.q4_pack(w, cb)
+        del w
+        packs.append((codes, scales, lin))
+        if lin.K not in xs:
+            xs[lin.K] = synth.activations_device(synth.x_seed(seed), 1, lin.K, dev)
+        ys.append(torch.empty((1, lin.N), dtype=torch.float32, device=dev))
+    torch.cuda.synchronize()
+    nbytes = sum(algo_bytes(1, lin.N, lin.K) for _, _, lin in packs)
+    with torch.cuda.stream(stream):
+        for (codes, scales, lin), y in zip(packs, ys):
+            q4.q4_gemv(codes, scales, cb, xs[lin.K], y)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for (codes, scales, lin), y in zip(packs, ys):
+            q4.q4_gemv(codes, scales, cb, xs[lin.K], y)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    del g, packs, xs, ys
+    torch.cuda.empty_cache()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": "llama31_8b_step: 32 x (qkv 4096->6144, o 4096->4096, gate_up 4096->28672, "
+                        "down 14336->4096) + lm_head 4096->128256, M=1, 129 q4_gemv launches in one "
+                        "CUDA graph",
+            "bytes_per_step": nbytes, "ms_per_step": round(ms, 4), "tok_s": round(1e3 / ms, 1),
+            "gbs": round(gbs, 1), "hbm_frac_of_measured": round(gbs / hbm_peak, 4)}
+
+
+def bench_small_m(dev, cb, stream, hbm_peak, Ms=(2, 4, 8, 16), reps=20):
+    """Verify batches on the Llama-3.1-8B linears + lm_head (396 MB packed, more
+    than L2, so each step streams its weights from HBM): q4_gemm of the five
+    linears at M tokens in one CUDA graph."""
+    import torch
+    import weight_only_bit_gemv_b200 as q4
+    wl = synth.WORKLOADS["small_m_verify"]
+    packs = []
+    for lin in wl.linears:
+        seed = synth.seed_for(wl.index, 0, lin.name)
+        w = synth.weights_device(seed, lin.N, lin.K, wl.w_std, dev)
+        codes, scales = q4.q4_pack(w, cb)
+        del w
+        packs.append((codes, scales, lin, seed))
+    out = {}
+    for M in Ms:
+        xs = [synth.activations_device(synth.x_seed(seed) + M, M, lin.K, dev) for _, _, lin, seed in packs]
+        ys = [torch.empty((M, lin.N), dtype=torch.float32, device=dev) for _, _, lin, _ in packs]
+        with torch.cuda.stream(stream):
+            for (codes, scales, lin, _), x, y in zip(packs, xs, ys):
+                q4.q4_gemm(codes, scales, cb, x, y)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for (codes, scales, lin, _), x, y in zip(packs, xs, ys):
+                q4.q4_gemm(codes, scales, cb, x, y)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g.replay()
+            e0.record()
+            for _ in range(reps):
+                g.replay()
+            e1.record()
+        e1.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        nbytes = sum(algo_bytes(M, lin.N, lin.K) for _, _, lin, _ in packs)
+        flops = sum(2.0 * M * lin.N * lin.K for _, _, lin, _ in packs)
+        out[f"M={M}"] = {"us": round(ms * 1e3, 2), "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                         "hbm_frac_of_measured": round(nbytes / (ms * 1e-3) / 1e9 / hbm_peak, 4),
+                         "tflops": round(flops / (ms * 1e-3) / 1e12, 2)}
+        del g, xs, ys
+    del packs
+    torch.cuda.empty_cache()
+    return {"workload": "small_m_verify: Llama-3.1-8B qkv, o, gate_up, down + lm_head, q4_gemm per "
+                        "linear, 5 launches in one CUDA graph", **out}
 
 
 def cpu_baseline(lins, cb, seconds):
@@ -531,6 +639,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-gemm", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-step", action="store_true", help="skip the Llama-3.1-8B decode step")
+    ap.add_argument("--no-smallm", action="store_true", help="skip the small-M verify batches")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     args = ap.parse_args()

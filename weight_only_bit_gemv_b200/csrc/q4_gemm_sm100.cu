@@ -16,20 +16,26 @@
 //
 // Roles (one CTA per tile of 128 weight rows x BMT tokens x one K chunk):
 //  * warp 0 streams, by TMA, stages of 4 groups of codes (a 128-row x
-//    128-byte box, 128-byte swizzle) with their scales (cp.async), and for
-//    every group the x tile (BMT tokens x 64 k binary16, 128-byte swizzle).
+//    128-byte box, 128-byte swizzle) with their scales (cp.async);
+//  * warp 10 streams, by TMA, the x tile of every group (BMT tokens x 64 k
+//    binary16, 128-byte swizzle) into the x stage of the group's ring slot;
 //  * warps 2-9 rebuild the weights: thread t of warp w owns row 32 (w mod 4) +
 //    t (its tensor-memory lane); per group it reads its 32 code bytes, looks
 //    each up in a 256-entry byte -> (cb[lo], cb[hi]) table (one copy per
 //    lane), multiplies by the scale with one HMUL2 and writes the 64 weights
-//    with one tcgen05.st into one of four A slots.  Even and odd groups go to
-//    the two halves of these warps.
+//    with one tcgen05.st into the A slot of the group's ring slot.  Even and
+//    odd groups go to the two halves of these warps.
 //  * warp 1 owns the tensor memory and, per group, issues four tcgen05.mma
 //    M=128 N=BMT K=16 (A from tensor memory, B = x tile from shared memory)
-//    into one fp32 accumulator of BMT columns; commits free the A slot and
-//    the x slot, and a last commit marks the accumulator ready.
+//    into one fp32 accumulator of BMT columns, then one commit that frees the
+//    group's ring slot (A slot and x stage together); a last commit marks the
+//    accumulator ready.
 //  * warps 2-9 then read the accumulator (tcgen05.ld) and write y, or add it
 //    into y with red.add when K is split across CTAs (y zeroed first).
+// Measured on B200: with one thread issuing the MMAs, an x stream tied to the
+// weight stream and two commits per group, that thread spent most of each
+// group waiting for x and committing; the separate x warp and the shared
+// ring (one commit) keep the tensor pipe fed.
 // Every wait is bounded; a timeout sets an error bit, the roles drain what
 // they have in flight and the CTA frees its tensor memory before it exits.
 #include <mutex>
@@ -49,9 +55,12 @@ constexpr int kWCodeBytes = kR * 128;     // one code box
 constexpr int kWScaleBytes = kR * 8;      // 4 scales per row
 constexpr int kLutBytes = 65536;
 constexpr int kDecWarps = 8;
-constexpr int kThreads = (2 + kDecWarps) * 32;
+constexpr int kXWarp = 2 + kDecWarps;  // the x producer
+constexpr int kThreads = (3 + kDecWarps) * 32;
 constexpr int kASlots = 4;
-constexpr int kWStages = 3;
+constexpr int kWStages = 2;
+// The A slots and the x stages form one ring: the MMA warp's one commit per
+// group frees both.
 constexpr uint32_t kTmemCols = 512;
 __device__ __forceinline__ uint32_t a_col(int slot) { return 256u + 32u * slot; }
 
@@ -100,15 +109,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t base = smem_u32(smem);
     const uint32_t bars = base + p.bar_off;
-    const int SX = p.xstages;
-    // barriers: wfull[2], wempty[2], xfull[SX], xempty[SX], afull[4], afree[4], dfull, cbbar, drain
+    // barriers: wfull, wempty [kWStages]; xfull, afull, gdone [kASlots]; dfull, cbbar, drain
     auto wfull = [&](int s) { return bars + 8u * s; };
     auto wempty = [&](int s) { return bars + 8u * (kWStages + s); };
     auto xfull = [&](int s) { return bars + 8u * (2 * kWStages + s); };
-    auto xempty = [&](int s) { return bars + 8u * (2 * kWStages + SX + s); };
-    auto afull = [&](int s) { return bars + 8u * (2 * kWStages + 2 * SX + s); };
-    auto afree = [&](int s) { return bars + 8u * (2 * kWStages + 2 * SX + kASlots + s); };
-    const uint32_t dfull = bars + 8u * (2 * kWStages + 2 * SX + 2 * kASlots);
+    auto afull = [&](int s) { return bars + 8u * (2 * kWStages + kASlots + s); };
+    auto gdone = [&](int s) { return bars + 8u * (2 * kWStages + 2 * kASlots + s); };
+    const uint32_t dfull = bars + 8u * (2 * kWStages + 3 * kASlots);
     const uint32_t cbbar = dfull + 8u;
     const uint32_t drain = dfull + 16u;
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + p.cb_off + 32);
@@ -128,13 +135,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(wfull(s), 33);  // expect_tx + one arrival per producer lane
             mbar_init(wempty(s), kDecWarps);
         }
-        for (int s = 0; s < SX; ++s) {
-            mbar_init(xfull(s), 1);
-            mbar_init(xempty(s), 1);  // tcgen05.commit
-        }
         for (int s = 0; s < kASlots; ++s) {
+            mbar_init(xfull(s), 1);   // expect_tx
             mbar_init(afull(s), 4);   // the four warps of the owning warpgroup
-            mbar_init(afree(s), 1);   // tcgen05.commit
+            mbar_init(gdone(s), 1);   // tcgen05.commit after the group's MMAs
         }
         mbar_init(dfull, 1);
         mbar_init(cbbar, 1);
@@ -155,11 +159,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------ producer ------------------------------
         if (lane == 0) {
             prefetch_tensor_map(&cmap);
-            prefetch_tensor_map(&xmap);
             mbar_arrive_expect_tx(cbbar, 32u);
             bulk_load(base + p.cb_off, p.cb, 32u, cbbar);
         }
-        int wi = 0, xi = 0;  // weight stages and x tiles issued
+        int wi = 0;  // weight stages issued
         bool ok = true;
         for (int w = 0; w < nw && ok; ++w) {
             // weight stage w: groups g_begin + 4w .. +3
@@ -198,22 +201,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             else
                 mbar_arrive(wfull(ws));
             ++wi;
-            // x tiles of these groups
-            for (int j = 0; j < kWG && ok; ++j) {
-                const int g = g0 + j;
-                if (g >= g_end) break;
-                const int xs = xi % SX;
-                if (xi >= SX && !warp_wait(xempty(xs), static_cast<uint32_t>(xi / SX - 1) & 1u, lane)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(xfull(xs), static_cast<uint32_t>(p.xstage_bytes));
-                    tma_load_2d(base + p.x_off + xs * p.xstage_bytes, &xmap, g * 64, tt * p.BMT, xfull(xs));
-                }
-                __syncwarp();
-                ++xi;
-            }
         }
         if (!ok && lane == 0) {
             atomicOr(&g_gemm_tc_error, 1u);
@@ -222,26 +209,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         // leave only once every copy issued has landed (bounded)
         for (int i = (wi > kWStages ? wi - kWStages : 0); i < wi; ++i)
             if (!warp_wait(wfull(i % kWStages), static_cast<uint32_t>(i / kWStages) & 1u, lane)) break;
-        for (int i = (xi > SX ? xi - SX : 0); i < xi; ++i)
-            if (!warp_wait(xfull(i % SX), static_cast<uint32_t>(i / SX) & 1u, lane)) break;
+    } else if (warp == kXWarp) {
+        // ----------------------------- x producer -----------------------------
+        // x tile of group gi -> ring slot gi mod kASlots, reused once the
+        // MMAs of group gi - kASlots are done.
+        if (lane == 0) prefetch_tensor_map(&xmap);
+        int xi = 0;
+        bool ok = true;
+        for (; xi < ng; ++xi) {
+            const int xs = xi % kASlots;
+            if (xi >= kASlots &&
+                !warp_wait(gdone(xs), static_cast<uint32_t>(xi / kASlots - 1) & 1u, lane)) {
+                ok = false;
+                break;
+            }
+            if (__shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(xfull(xs), static_cast<uint32_t>(p.xstage_bytes));
+                tma_load_2d(base + p.x_off + xs * p.xstage_bytes, &xmap, (g_begin + xi) * 64, tt * p.BMT,
+                            xfull(xs));
+            }
+            __syncwarp();
+        }
+        if (!ok && lane == 0) {
+            atomicOr(&g_gemm_tc_error, 4u);
+            *abort_flag = 1;
+        }
+        for (int i = (xi > kASlots ? xi - kASlots : 0); i < xi; ++i)
+            if (!warp_wait(xfull(i % kASlots), static_cast<uint32_t>(i / kASlots) & 1u, lane)) break;
     } else if (warp == 1) {
         // -------------------------------- MMA ---------------------------------
         if (lane == 0) {
             bool ok = true;
             for (int gi = 0; gi < ng && ok; ++gi) {
-                const int as = gi % kASlots, xs = gi % SX;
+                const int as = gi % kASlots;
                 if (!mbar_wait(afull(as), static_cast<uint32_t>(gi / kASlots) & 1u) ||
-                    !mbar_wait(xfull(xs), static_cast<uint32_t>(gi / SX) & 1u) || *abort_flag) {
+                    !mbar_wait(xfull(as), static_cast<uint32_t>(gi / kASlots) & 1u) || *abort_flag) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint64_t bd = smem_desc_sw128(base + p.x_off + xs * p.xstage_bytes, 1024);
+                const uint64_t bd = smem_desc_sw128(base + p.x_off + as * p.xstage_bytes, 1024);
 #pragma unroll
                 for (int t = 0; t < 4; ++t)
                     tc_mma_ts(tmem, tmem + a_col(as) + 8 * t, bd + 2 * t, p.idesc, (gi > 0 || t > 0) ? 1u : 0u);
-                tc_commit(afree(as));
-                tc_commit(xempty(xs));
+                tc_commit(gdone(as));  // frees the A slot and the x stage
             }
             if (ok) tc_commit(dfull);
             if (!ok) {
@@ -278,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = false;
                 break;
             }
-            if (gi >= kASlots && !warp_wait(afree(as), static_cast<uint32_t>(gi / kASlots - 1) & 1u, lane)) {
+            if (gi >= kASlots && !warp_wait(gdone(as), static_cast<uint32_t>(gi / kASlots - 1) & 1u, lane)) {
                 ok = false;
                 break;
             }
@@ -414,15 +426,13 @@ cudaError_t launch_prefill_tc(const uint8_t* codes, const uint16_t* scales, cons
     p.idesc = idesc_f16_f32(kR, p.BMT);
     p.wscale_off = kLutBytes + kWStages * kWCodeBytes;
     p.x_off = (p.wscale_off + kWStages * kWScaleBytes + 1023) & ~1023;
-    const int fixed = p.x_off + 64 + 512 + 1024;
-    int SX = (dev.smem_optin - fixed) / p.xstage_bytes;
-    if (SX > 6) SX = 6;
-    if (SX < 2) return cudaErrorNotSupported;
+    const int SX = kASlots;  // one x stage per A slot
     p.xstages = SX;
     p.cb_off = p.x_off + SX * p.xstage_bytes;
     p.bar_off = p.cb_off + 64;
-    const int nbars = 2 * kWStages + 2 * SX + 2 * kASlots + 3;
+    const int nbars = 2 * kWStages + 3 * kASlots + 3;
     const int smem = p.bar_off + nbars * 8;
+    if (smem > dev.smem_optin) return cudaErrorNotSupported;
 
     // x -> binary16 into the scratch buffer
     const int64_t n8 = M * K / 8;
