@@ -268,6 +268,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
         int slot = 0, t = 0, c = 0;
         uint32_t eparity = 1;  // parity of the empty phase to wait for (round - 1)
         for (int i = 0; i < total; ++i) {
+            if (i == 2) {
+                // let the first stage land before the rest of the ring is
+                // requested, so that it is not served behind them
+                uint32_t ok = 1;
+                if (lane == 0) ok = mbar_wait(bars, 0u) ? 1u : 0u;
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) {
+                    if (lane == 0) atomicOr(&g_gemv_m1_error, 0x200u);
+                    break;
+                }
+            }
             if (i >= NS) {
                 uint32_t ok = 1;
                 if (lane == 0) ok = mbar_wait(bars + 8u * (NS + slot), eparity) ? 1u : 0u;
@@ -328,7 +339,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
         // Issue every global read of the set-up at once (the codebook and all
         // of x: one 16-byte chunk per thread and round), then build the table
         // and the x layout: one memory latency instead of one per round.
-        const uint32_t cbv = p.cb[lane & 15];
+        // this thread's table entry b = tid: (cb[b & 15], cb[b >> 4])
+        const uint32_t ent = static_cast<uint32_t>(p.cb[tid & 15]) |
+                             (static_cast<uint32_t>(p.cb[tid >> 4]) << 16);
         const int nx = p.K >> 3;  // 16-byte chunks of x (8 values)
         uint4 xv[kXRounds];
 #pragma unroll
@@ -337,12 +350,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
             xv[i] = r < nx ? __ldg(reinterpret_cast<const uint4*>(p.x) + r) : make_uint4(0u, 0u, 0u, 0u);
         }
         asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
-        // byte -> (cb[lo], cb[hi]) table, one copy per lane
-        for (int b = warp; b < 256; b += kCW) {
-            const uint32_t lo = __shfl_sync(0xFFFFFFFFu, cbv, b & 15);
-            const uint32_t hi = __shfl_sync(0xFFFFFFFFu, cbv, b >> 4);
-            *reinterpret_cast<uint32_t*>(smem + b * 256 + lane * 4) = lo | (hi << 16);
-        }
+        // byte -> (cb[lo], cb[hi]) table, one copy per lane: thread tid writes
+        // the 32 copies of entry tid, four per 16-byte store, starting at a
+        // lane-rotated chunk so that a store of the warp spreads over the banks
+        static_assert(kCW * 32 == 256, "one table entry per consumer thread");
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            *reinterpret_cast<uint4*>(smem + tid * 256 + 16 * ((i + lane) & 7)) =
+                make_uint4(ent, ent, ent, ent);
         // x as binary16: 16-byte chunk (span s, quarter q, parity par, j)
         // holds x[128 s + 32 j + 8 q, +8) when par == j / 2 (the column of
         // that group), else zeros; chunks past K are zeros.
