@@ -203,10 +203,12 @@ int q4_abi_version(void);
  * kernels is bounded (about two seconds); a wait that runs out sets a bit in
  * a device word, the kernel drains what it has in flight, frees its tensor
  * memory and exits, leaving its output incomplete.  This call synchronizes the
- * current device, stores the bits set since the last call in *flags (bits
- * 0-15: the M = 1 GEMV, bit 8 there meaning that its shared-memory layout did
- * not match the device; bits 16-31: the M > 16 tensor-core GEMM; 0 = none)
- * and clears them.  Not an operation of the method; a health check.
+ * current device, stores the bits set since the last call in *flags and
+ * clears them: bits 0-11 the M = 1 GEMV (bit 8: its shared-memory layout did
+ * not match the device; bits 9-11: producer, drain and consumer waits), bits
+ * 12-15 the M = 2..16 kernel (the same four conditions), bits 16-31 the
+ * M > 16 tensor-core GEMM; 0 = none.  Not an operation of the method; a
+ * health check.
  * Returns Q4_ERR_NULL for a NULL flags, Q4_ERR_CUDA if a CUDA call fails.
  */
 q4_status q4_timeout_flags(uint32_t* flags);

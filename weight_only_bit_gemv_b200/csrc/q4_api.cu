@@ -212,11 +212,12 @@ int q4_abi_version(void) { return Q4_ABI_VERSION; }
 q4_status q4_timeout_flags(uint32_t* flags) {
     if (!flags) return Q4_ERR_NULL;
     *flags = 0;
-    unsigned int a = 0, b = 0;
+    unsigned int a = 0, b = 0, c = 0;
     cudaError_t e = take_gemv_m1_error(&a);
     if (e == cudaSuccess) e = take_gemm_tc_error(&b);
+    if (e == cudaSuccess) e = take_gemm_small_error(&c);
     if (e != cudaSuccess) return cuda_fail(e);
-    *flags = (a & 0xFFFFu) | ((b & 0xFFFFu) << 16);
+    *flags = (a & 0x0FFFu) | ((c & 0x0F00u) << 4) | ((b & 0xFFFFu) << 16);
     return Q4_OK;
 }
 

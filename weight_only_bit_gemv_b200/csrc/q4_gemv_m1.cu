@@ -62,12 +62,14 @@ constexpr int kSpan = 128;                // k per span (64 code bytes)
 constexpr int kMaxKC = 2048;              // code bytes of a row per stage
 constexpr int kPassTiles = 128;           // tiles per pass of the shared row accumulator
 constexpr int kAhead = 3;                 // scale prefetch distance, in stages
-constexpr int kMaxStages = 6;
+constexpr int kMaxStages = 6;  // 2 * kMaxStages barriers fit below kDepOff
 constexpr int kXEmbedSpans = 64;          // spans whose x fits in the table rows' free halves
 constexpr int kXRounds = 13;              // x chunk loads per consumer thread: K <= 13 * 256 * 8
 constexpr uint32_t kAccOff = kLutBytes;
 constexpr uint32_t kBarOff = kAccOff + kPassTiles * 16 * 4;
 constexpr uint32_t kXOff = kBarOff + 128;
+constexpr uint32_t kDepOff = kXOff - 4;   // past the 2 * kMaxStages barriers
+static_assert(kBarOff + 2 * kMaxStages * 8 <= kDepOff, "barriers overlap the dependency word");
 
 struct M1 {
     const uint8_t* codes;
@@ -81,6 +83,7 @@ struct M1 {
     int KC;          // code bytes of a row per stage (the ring's row pitch)
     int C;           // stages per 16-row tile
     int NS;          // ring stages
+    int early;       // weights static: read them before waiting for the preceding kernel
     uint32_t ring_off, stage_bytes;
 };
 
@@ -90,6 +93,15 @@ struct M1 {
 __device__ __forceinline__ uint32_t ldg_u32(const void* p) {
     uint32_t v;
     asm("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+// A load that stays under the branch that guards it (never hoisted).
+__device__ __forceinline__ uint4 ldg_v4_ordered(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
     return v;
 }
 
@@ -233,61 +245,36 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
         }
         fence_mbar_init();
     }
-    // Warm L2 with the first stage while the preceding kernel finishes (more
-    // would queue ahead of the set-up's reads of x in DRAM).
-    if (warp == kCW) {
-        for (int i = 0; i < 1 && i < total; ++i) {
-            const int t = i / p.C, c = i - t * p.C;
-            const int rows = min(16, nrows - 16 * t);
+    // x may be written by the preceding kernel: before the wait it is only
+    // prefetched into L2 (a prefetch is coherent, L2 being the point of
+    // coherence), so the reads after the wait find it there.
+    if (warp == kCW && lane == 30) prefetch_l2(p.x, static_cast<uint32_t>(p.K) * 2u);
+    if (!p.early) {
+        // Warm L2 with the first stage and its scales while the preceding
+        // kernel finishes (more would queue ahead of the reads of x).
+        if (warp == kCW && total > 0) {
+            const int rows = min(16, nrows);
             if (kWhole) {
                 if (lane == 0)
-                    prefetch_l2(p.codes + static_cast<int64_t>(r0 + 16 * t) * p.rowbytes,
+                    prefetch_l2(p.codes + static_cast<int64_t>(r0) * p.rowbytes,
                                 static_cast<uint32_t>(rows * p.rowbytes));
             } else if (lane < rows) {
-                prefetch_l2(p.codes + static_cast<int64_t>(r0 + 16 * t + lane) * p.rowbytes + c * p.KC,
-                            static_cast<uint32_t>(min(p.KC, p.rowbytes - c * p.KC)));
+                prefetch_l2(p.codes + static_cast<int64_t>(r0 + lane) * p.rowbytes,
+                            static_cast<uint32_t>(min(p.KC, p.rowbytes)));
             }
         }
+        if (warp == kCW && lane == 31)
+            prefetch_scales_l2(p.scales, p.G, p.N, r0, r0 + min(nrows, 32));
+        if (warp == kCW && lane == 29) prefetch_l2(p.cb, 32u);
     }
-    if (warp == kCW && lane == 31)
-        prefetch_scales_l2(p.scales, p.G, p.N, r0, r0 + min(nrows, 32));
-    // x and the codebook too: a prefetch is coherent (L2 is the point of
-    // coherence), so this is safe even if the preceding kernel writes them;
-    // the reads below, after the wait, then find them in L2.
-    if (warp == kCW && lane == 30) prefetch_l2(p.x, static_cast<uint32_t>(p.K) * 2u);
-    if (warp == kCW && lane == 29) prefetch_l2(p.cb, 32u);
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     __syncthreads();
 
     if (warp == kCW) {
         // ------------------------------ producer ------------------------------
-        // The set-up's reads of x and the codebook go out first; the weight
-        // stream starts once every consumer has issued them.
-        asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
         const uint32_t ring = base + p.ring_off;
         int slot = 0, t = 0, c = 0;
         uint32_t eparity = 1;  // parity of the empty phase to wait for (round - 1)
-        for (int i = 0; i < total; ++i) {
-            if (i == 2) {
-                // let the first stage land before the rest of the ring is
-                // requested, so that it is not served behind them
-                uint32_t ok = 1;
-                if (lane == 0) ok = mbar_wait(bars, 0u) ? 1u : 0u;
-                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-                if (!ok) {
-                    if (lane == 0) atomicOr(&g_gemv_m1_error, 0x200u);
-                    break;
-                }
-            }
-            if (i >= NS) {
-                uint32_t ok = 1;
-                if (lane == 0) ok = mbar_wait(bars + 8u * (NS + slot), eparity) ? 1u : 0u;
-                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-                if (!ok) {
-                    if (lane == 0) atomicOr(&g_gemv_m1_error, 0x200u);
-                    break;
-                }
-            }
+        auto issue = [&]() {
             const int rows = min(16, nrows - 16 * t);
             const uint32_t dst = ring + slot * p.stage_bytes;
             const uint32_t full = bars + 8u * slot;
@@ -321,6 +308,45 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
                 slot = 0;
                 eparity ^= 1u;
             }
+        };
+        int i = 0;
+        if (p.early) {
+            // Static weights: the first stage is copied while the preceding
+            // kernel finishes.  The rest of the ring waits until every
+            // consumer holds its x, so that x is not served behind it.
+            if (total > 0) {
+                issue();
+                i = 1;
+            }
+            asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
+        } else {
+            // The set-up's reads of x and the codebook go out first; the
+            // weight stream starts once every consumer has issued them.
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
+        }
+        for (; i < total; ++i) {
+            if (i == 2) {
+                // let the first stage land before the rest of the ring is
+                // requested, so that it is not served behind them
+                uint32_t ok = 1;
+                if (lane == 0) ok = mbar_wait(bars, 0u) ? 1u : 0u;
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) {
+                    if (lane == 0) atomicOr(&g_gemv_m1_error, 0x200u);
+                    break;
+                }
+            }
+            if (i >= NS) {
+                uint32_t ok = 1;
+                if (lane == 0) ok = mbar_wait(bars + 8u * (NS + slot), eparity) ? 1u : 0u;
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) {
+                    if (lane == 0) atomicOr(&g_gemv_m1_error, 0x200u);
+                    break;
+                }
+            }
+            issue();
         }
         // Leave only once this warp's copies have landed (bounded).
         if (lane == 0) {
@@ -335,59 +361,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
 
     // ------------------------------- consumers ------------------------------
     float* acc_s = reinterpret_cast<float*>(smem + kAccOff);
-    {
-        // Issue every global read of the set-up at once (the codebook and all
-        // of x: one 16-byte chunk per thread and round), then build the table
-        // and the x layout: one memory latency instead of one per round.
-        // this thread's table entry b = tid: (cb[b & 15], cb[b >> 4])
-        const uint32_t ent = static_cast<uint32_t>(p.cb[tid & 15]) |
-                             (static_cast<uint32_t>(p.cb[tid >> 4]) << 16);
-        const int nx = p.K >> 3;  // 16-byte chunks of x (8 values)
-        uint4 xv[kXRounds];
-#pragma unroll
-        for (int i = 0; i < kXRounds; ++i) {
-            const int r = tid + i * kCW * 32;
-            xv[i] = r < nx ? __ldg(reinterpret_cast<const uint4*>(p.x) + r) : make_uint4(0u, 0u, 0u, 0u);
-        }
-        asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
-        // byte -> (cb[lo], cb[hi]) table, one copy per lane: thread tid writes
-        // the 32 copies of entry tid, four per 16-byte store, starting at a
-        // lane-rotated chunk so that a store of the warp spreads over the banks
-        static_assert(kCW * 32 == 256, "one table entry per consumer thread");
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            *reinterpret_cast<uint4*>(smem + tid * 256 + 16 * ((i + lane) & 7)) =
-                make_uint4(ent, ent, ent, ent);
-        // x as binary16: 16-byte chunk (span s, quarter q, parity par, j)
-        // holds x[128 s + 32 j + 8 q, +8) when par == j / 2 (the column of
-        // that group), else zeros; chunks past K are zeros.
-        auto chunk_off = [&](int s, int q, int par, int j) -> uint32_t {
-            return kXEmb ? (4 * s + q) * 256 + 128 + par * 64 + j * 16
-                         : kXOff + s * 512 + q * 128 + par * 64 + j * 16;
-        };
-#pragma unroll
-        for (int i = 0; i < kXRounds; ++i) {
-            const int r = tid + i * kCW * 32;
-            if (r < nx) {
-                const int k = 8 * r;
-                const int s = k >> 7, j = (k >> 5) & 3, q = (k >> 3) & 3;
-                uint4 h;
-                h.x = cvt_bf16x2_f16x2(xv[i].x);
-                h.y = cvt_bf16x2_f16x2(xv[i].y);
-                h.z = cvt_bf16x2_f16x2(xv[i].z);
-                h.w = cvt_bf16x2_f16x2(xv[i].w);
-                *reinterpret_cast<uint4*>(smem + chunk_off(s, q, j >> 1, j)) = h;
-                *reinterpret_cast<uint4*>(smem + chunk_off(s, q, 1 - (j >> 1), j)) =
-                    make_uint4(0u, 0u, 0u, 0u);
-            }
-        }
-        // the spans that reach past K: their chunks beyond K are zeros
-        for (int c = (p.S - 1) * 32 + tid; c < p.SP * 32; c += kCW * 32) {
-            const int j = c & 3, par = (c >> 2) & 1, q = (c >> 3) & 3, s = c >> 5;
-            if (s * kSpan + 32 * j + 8 * q >= p.K)
-                *reinterpret_cast<uint4*>(smem + chunk_off(s, q, par, j)) = make_uint4(0u, 0u, 0u, 0u);
-        }
-    }
     constexpr uint32_t kXSpan = kXEmb ? 1024u : 512u;  // x bytes between spans
     const int upk = p.KC >> 7;                         // units (256 k) per full stage
     // this lane's code offsets in a stage: rows g and g + 8, pass A and B
@@ -426,9 +399,122 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
             }
         }
     };
-    scale_rows();
+
+    // this thread's table entry b = tid: (cb[b & 15], cb[b >> 4])
+    static_assert(kCW * 32 == 256, "one table entry per consumer thread");
+    auto cb_entry = [&]() -> uint32_t {
+        return static_cast<uint32_t>(p.cb[tid & 15]) | (static_cast<uint32_t>(p.cb[tid >> 4]) << 16);
+    };
+    // byte -> (cb[lo], cb[hi]) table, one copy per lane: thread tid writes the
+    // 32 copies of entry tid, four per 16-byte store, starting at a
+    // lane-rotated chunk so that a store of the warp spreads over the banks
+    auto build_table = [&](uint32_t ent) {
 #pragma unroll
-    for (int i = 0; i < kAhead; ++i) next_scales(sc[i]);
+        for (int i = 0; i < 8; ++i)
+            *reinterpret_cast<uint4*>(smem + tid * 256 + 16 * ((i + lane) & 7)) =
+                make_uint4(ent, ent, ent, ent);
+    };
+    uint32_t xw[kUPW][16];  // whole rows: this warp's units never change, nor their x
+    if (p.early) {
+        build_table(cb_entry());
+        scale_rows();
+#pragma unroll
+        for (int i = 0; i < kAhead; ++i) next_scales(sc[i]);
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    {
+        // Issue every global read of the set-up at once, then build the table
+        // and x: one memory latency instead of one per round.
+        const uint32_t ent = p.early ? 0u : cb_entry();
+        const int nx = p.K >> 3;  // 16-byte chunks of x (8 values)
+        uint4 xv[kXRounds];
+        if (kWhole) {
+            // The B fragments of this warp's units U = warp + kCW j straight
+            // from x, in the column layout the shared-memory copy has
+            // otherwise: lane (g, tq) holds x[128 s + 32 tq, +32) of span
+            // s = 2 U + (g / 2) % 2 when g % 2 == tq / 2, else zeros.
+#pragma unroll
+            for (int j = 0; j < kUPW; ++j) {
+                const int U = warp + kCW * j;
+                const bool act = U < upk && (g & 1) == (tq >> 1);
+                const uint16_t* xs = p.x + kSpan * (2 * U + ((g >> 1) & 1)) + 32 * tq;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (act) v = ldg_v4_ordered(xs + 8 * q);
+                    xw[j][4 * q] = v.x;
+                    xw[j][4 * q + 1] = v.y;
+                    xw[j][4 * q + 2] = v.z;
+                    xw[j][4 * q + 3] = v.w;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < kXRounds; ++i) {
+                const int r = tid + i * kCW * 32;
+                xv[i] = r < nx ? __ldg(reinterpret_cast<const uint4*>(p.x) + r)
+                               : make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        if (!p.early) {
+            asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
+            build_table(ent);
+        }
+        uint32_t dep = 0;  // depends on every x value this thread loaded
+        if (kWhole) {
+#pragma unroll
+            for (int j = 0; j < kUPW; ++j)
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    dep |= xw[j][i];
+                    xw[j][i] = cvt_bf16x2_f16x2(xw[j][i]);
+                }
+        } else {
+            // x as binary16: 16-byte chunk (span s, quarter q, parity par, j)
+            // holds x[128 s + 32 j + 8 q, +8) when par == j / 2 (the column
+            // of that group), else zeros; chunks past K are zeros.
+            auto chunk_off = [&](int s, int q, int par, int j) -> uint32_t {
+                return kXEmb ? (4 * s + q) * 256 + 128 + par * 64 + j * 16
+                             : kXOff + s * 512 + q * 128 + par * 64 + j * 16;
+            };
+#pragma unroll
+            for (int i = 0; i < kXRounds; ++i) {
+                const int r = tid + i * kCW * 32;
+                dep |= xv[i].x;
+                if (r < nx) {
+                    const int k = 8 * r;
+                    const int s = k >> 7, j = (k >> 5) & 3, q = (k >> 3) & 3;
+                    uint4 h;
+                    h.x = cvt_bf16x2_f16x2(xv[i].x);
+                    h.y = cvt_bf16x2_f16x2(xv[i].y);
+                    h.z = cvt_bf16x2_f16x2(xv[i].z);
+                    h.w = cvt_bf16x2_f16x2(xv[i].w);
+                    *reinterpret_cast<uint4*>(smem + chunk_off(s, q, j >> 1, j)) = h;
+                    *reinterpret_cast<uint4*>(smem + chunk_off(s, q, 1 - (j >> 1), j)) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            // the spans that reach past K: their chunks beyond K are zeros
+            for (int c = (p.S - 1) * 32 + tid; c < p.SP * 32; c += kCW * 32) {
+                const int j = c & 3, par = (c >> 2) & 1, q = (c >> 3) & 3, s = c >> 5;
+                if (s * kSpan + 32 * j + 8 * q >= p.K)
+                    *reinterpret_cast<uint4*>(smem + chunk_off(s, q, par, j)) =
+                        make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        // Static weights: the producer requests the rest of the ring once
+        // every consumer's x has arrived.  The store of `dep` cannot issue
+        // before the loads have returned, and the arrival issues after it.
+        if (p.early) {
+            *reinterpret_cast<volatile uint32_t*>(smem + kDepOff) = dep;
+            asm volatile("bar.arrive 2, %0;" ::"n"(kThreads) : "memory");
+        }
+    }
+    if (!p.early) {
+        scale_rows();
+#pragma unroll
+        for (int i = 0; i < kAhead; ++i) next_scales(sc[i]);
+    }
 
     // One unit: two passes of eight MMAs; lane tq in {0, 1} adds span
     // 2U + tq of rows g and g + 8, each group scaled by its own scale.
@@ -470,7 +556,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
 
     bool started = false;
     uint32_t xlane = 0;
-    uint32_t xw[kUPW][16];  // whole rows: this warp's units never change, nor their x
     int slot = 0;
     uint32_t fparity = 0;
     for (int pt0 = 0; pt0 < T; pt0 += kPassTiles) {
@@ -482,11 +567,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
             // x read below it
             xlane = base + (kXEmb ? 128u : kXOff) + ((g >> 1) & 1) * kXSpan + (g & 1) * 64 + tq * 16;
             asm volatile("" : "+r"(xlane)::"memory");
-            if (kWhole) {
-#pragma unroll
-                for (int j = 0; j < kUPW; ++j)
-                    load_x(xlane + static_cast<uint32_t>(warp + kCW * j) * (2 * kXSpan), xw[j]);
-            }
             started = true;
         }
         for (int t = pt0; t < pt1; ++t) {
@@ -572,9 +652,10 @@ cudaError_t take_gemv_m1_error(unsigned int* out) {
 
 cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
-                           const DeviceInfo& dev) {
+                           const DeviceInfo& dev, bool weights_static) {
     if (dev.smem_reserved != kBase) return cudaErrorNotSupported;
     M1 p{};
+    p.early = weights_static ? 1 : 0;
     p.codes = codes;
     p.scales = scales;
     p.cb = cb;
