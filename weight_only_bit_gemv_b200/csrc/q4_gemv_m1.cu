@@ -34,9 +34,11 @@
 //    outside its group, so one chain of eight MMAs per pass yields every
 //    row's per-group sums in columns 0-3; lane tq in {0, 1} keeps span
 //    2u + tq of its rows and scales each group's fp32 sum by its own scale.
-//  * x is rounded to binary16 once per CTA into shared memory in that
-//    column layout (for K <= 8192 inside the unused half of the table rows).
-//    Scales are read from global memory by the consumers, stages ahead.
+//  * x is rounded to binary16 once per CTA.  When a tile is one stage, each
+//    warp loads its units' B fragments straight into registers for the whole
+//    kernel; otherwise x goes to shared memory in that column layout (for
+//    K <= 8192 inside the unused half of the table rows).  Scales are read
+//    from global memory by the consumers, stages ahead.
 //  * The warps of a CTA add their tile sums into a shared-memory row
 //    accumulator; the CTA writes each y element once (no split-K between
 //    CTAs, no zeroing of y, no global atomics).
@@ -62,14 +64,13 @@ constexpr int kSpan = 128;                // k per span (64 code bytes)
 constexpr int kMaxKC = 2048;              // code bytes of a row per stage
 constexpr int kPassTiles = 128;           // tiles per pass of the shared row accumulator
 constexpr int kAhead = 3;                 // scale prefetch distance, in stages
-constexpr int kMaxStages = 6;  // 2 * kMaxStages barriers fit below kDepOff
+constexpr int kMaxStages = 6;
 constexpr int kXEmbedSpans = 64;          // spans whose x fits in the table rows' free halves
 constexpr int kXRounds = 13;              // x chunk loads per consumer thread: K <= 13 * 256 * 8
 constexpr uint32_t kAccOff = kLutBytes;
 constexpr uint32_t kBarOff = kAccOff + kPassTiles * 16 * 4;
 constexpr uint32_t kXOff = kBarOff + 128;
-constexpr uint32_t kDepOff = kXOff - 4;   // past the 2 * kMaxStages barriers
-static_assert(kBarOff + 2 * kMaxStages * 8 <= kDepOff, "barriers overlap the dependency word");
+static_assert(2 * kMaxStages * 8 <= 128, "barriers overflow their area");
 
 struct M1 {
     const uint8_t* codes;
@@ -83,7 +84,6 @@ struct M1 {
     int KC;          // code bytes of a row per stage (the ring's row pitch)
     int C;           // stages per 16-row tile
     int NS;          // ring stages
-    int early;       // weights static: read them before waiting for the preceding kernel
     uint32_t ring_off, stage_bytes;
 };
 
@@ -249,24 +249,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
     // prefetched into L2 (a prefetch is coherent, L2 being the point of
     // coherence), so the reads after the wait find it there.
     if (warp == kCW && lane == 30) prefetch_l2(p.x, static_cast<uint32_t>(p.K) * 2u);
-    if (!p.early) {
-        // Warm L2 with the first stage and its scales while the preceding
-        // kernel finishes (more would queue ahead of the reads of x).
-        if (warp == kCW && total > 0) {
-            const int rows = min(16, nrows);
-            if (kWhole) {
-                if (lane == 0)
-                    prefetch_l2(p.codes + static_cast<int64_t>(r0) * p.rowbytes,
-                                static_cast<uint32_t>(rows * p.rowbytes));
-            } else if (lane < rows) {
-                prefetch_l2(p.codes + static_cast<int64_t>(r0 + lane) * p.rowbytes,
-                            static_cast<uint32_t>(min(p.KC, p.rowbytes)));
-            }
+    // Warm L2 with the first stage and its scales while the preceding kernel
+    // finishes (more would queue ahead of the reads of x).
+    if (warp == kCW && total > 0) {
+        const int rows = min(16, nrows);
+        if (kWhole) {
+            if (lane == 0)
+                prefetch_l2(p.codes + static_cast<int64_t>(r0) * p.rowbytes,
+                            static_cast<uint32_t>(rows * p.rowbytes));
+        } else if (lane < rows) {
+            prefetch_l2(p.codes + static_cast<int64_t>(r0 + lane) * p.rowbytes,
+                        static_cast<uint32_t>(min(p.KC, p.rowbytes)));
         }
-        if (warp == kCW && lane == 31)
-            prefetch_scales_l2(p.scales, p.G, p.N, r0, r0 + min(nrows, 32));
-        if (warp == kCW && lane == 29) prefetch_l2(p.cb, 32u);
     }
+    if (warp == kCW && lane == 31) prefetch_scales_l2(p.scales, p.G, p.N, r0, r0 + min(nrows, 32));
+    if (warp == kCW && lane == 29) prefetch_l2(p.cb, 32u);
     __syncthreads();
 
     if (warp == kCW) {
@@ -309,23 +306,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
                 eparity ^= 1u;
             }
         };
-        int i = 0;
-        if (p.early) {
-            // Static weights: the first stage is copied while the preceding
-            // kernel finishes.  The rest of the ring waits until every
-            // consumer holds its x, so that x is not served behind it.
-            if (total > 0) {
-                issue();
-                i = 1;
-            }
-            asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
-        } else {
-            // The set-up's reads of x and the codebook go out first; the
-            // weight stream starts once every consumer has issued them.
-            asm volatile("griddepcontrol.wait;" ::: "memory");
-            asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
-        }
-        for (; i < total; ++i) {
+        // The set-up's reads of x and the codebook go out first; the weight
+        // stream starts once every consumer has issued them.
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
+        for (int i = 0; i < total; ++i) {
             if (i == 2) {
                 // let the first stage land before the rest of the ring is
                 // requested, so that it is not served behind them
@@ -415,17 +400,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
                 make_uint4(ent, ent, ent, ent);
     };
     uint32_t xw[kUPW][16];  // whole rows: this warp's units never change, nor their x
-    if (p.early) {
-        build_table(cb_entry());
-        scale_rows();
-#pragma unroll
-        for (int i = 0; i < kAhead; ++i) next_scales(sc[i]);
-    }
     asm volatile("griddepcontrol.wait;" ::: "memory");
     {
         // Issue every global read of the set-up at once, then build the table
         // and x: one memory latency instead of one per round.
-        const uint32_t ent = p.early ? 0u : cb_entry();
+        const uint32_t ent = cb_entry();
         const int nx = p.K >> 3;  // 16-byte chunks of x (8 values)
         uint4 xv[kXRounds];
         if (kWhole) {
@@ -456,19 +435,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
                                : make_uint4(0u, 0u, 0u, 0u);
             }
         }
-        if (!p.early) {
-            asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
-            build_table(ent);
-        }
-        uint32_t dep = 0;  // depends on every x value this thread loaded
+        asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
+        build_table(ent);
         if (kWhole) {
 #pragma unroll
             for (int j = 0; j < kUPW; ++j)
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    dep |= xw[j][i];
-                    xw[j][i] = cvt_bf16x2_f16x2(xw[j][i]);
-                }
+                for (int i = 0; i < 16; ++i) xw[j][i] = cvt_bf16x2_f16x2(xw[j][i]);
         } else {
             // x as binary16: 16-byte chunk (span s, quarter q, parity par, j)
             // holds x[128 s + 32 j + 8 q, +8) when par == j / 2 (the column
@@ -480,7 +453,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
 #pragma unroll
             for (int i = 0; i < kXRounds; ++i) {
                 const int r = tid + i * kCW * 32;
-                dep |= xv[i].x;
                 if (r < nx) {
                     const int k = 8 * r;
                     const int s = k >> 7, j = (k >> 5) & 3, q = (k >> 3) & 3;
@@ -502,19 +474,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
                         make_uint4(0u, 0u, 0u, 0u);
             }
         }
-        // Static weights: the producer requests the rest of the ring once
-        // every consumer's x has arrived.  The store of `dep` cannot issue
-        // before the loads have returned, and the arrival issues after it.
-        if (p.early) {
-            *reinterpret_cast<volatile uint32_t*>(smem + kDepOff) = dep;
-            asm volatile("bar.arrive 2, %0;" ::"n"(kThreads) : "memory");
-        }
     }
-    if (!p.early) {
-        scale_rows();
+    scale_rows();
 #pragma unroll
-        for (int i = 0; i < kAhead; ++i) next_scales(sc[i]);
-    }
+    for (int i = 0; i < kAhead; ++i) next_scales(sc[i]);
 
     // One unit: two passes of eight MMAs; lane tq in {0, 1} adds span
     // 2U + tq of rows g and g + 8, each group scaled by its own scale.
@@ -652,10 +615,9 @@ cudaError_t take_gemv_m1_error(unsigned int* out) {
 
 cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
-                           const DeviceInfo& dev, bool weights_static) {
+                           const DeviceInfo& dev) {
     if (dev.smem_reserved != kBase) return cudaErrorNotSupported;
     M1 p{};
-    p.early = weights_static ? 1 : 0;
     p.codes = codes;
     p.scales = scales;
     p.cb = cb;

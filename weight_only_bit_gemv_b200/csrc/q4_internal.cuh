@@ -38,17 +38,15 @@ cudaError_t launch_pack(const float* w, const uint16_t* cb, uint8_t* codes, uint
 cudaError_t launch_dequant(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            float* w, int64_t N, int64_t K, cudaStream_t s, const DeviceInfo& dev);
 // M in [1, 16]: decoded codebook values on mma.sync, exact products, fp32 sums.
-// weights_static (M = 1 only): the weights may be read before the preceding
-// kernel on the stream has finished (see q4_gemv_ex).
 cudaError_t launch_small_m(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int M, int64_t N, int64_t K,
-                           cudaStream_t s, const DeviceInfo& dev, bool weights_static = false);
+                           cudaStream_t s, const DeviceInfo& dev);
 // M = 1: bulk-copy-fed decode GEMV, one row range per CTA, launched with
 // programmatic dependent launch.  Returns cudaErrorNotSupported when the
 // shape does not fit it (K too large for its shared-memory layout).
 cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
-                           const DeviceInfo& dev, bool weights_static);
+                           const DeviceInfo& dev);
 // M in [2, 16]: TMA-fed row blocks, decoded weights on mma.sync with the
 // tokens as B columns, exact products.  Returns cudaErrorNotSupported when the
 // device's shared-memory layout or the shape does not fit it.
