@@ -280,70 +280,76 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!bad) {
                 const uint32_t st = ring + slot * kStageBytes;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    if (kb + 256 * h >= kend) break;
+                // group j of the stage: box j / 4, group j % 4 of the box
+                auto group = [&](int j) {
+                    const int h = j >> 2, gm = j & 3;
                     const uint32_t box = st + h * kBoxBytes;
+                    const int kk = kb + 64 * j;  // first k of the group
+                    // 8 code bytes of the group for each row: 16-byte chunk
+                    // 2 gm + tq / 2 of the row, swizzled by the row (rho < 8)
+                    const uint32_t off =
+                        (static_cast<uint32_t>((2 * gm + (tq >> 1)) ^ rho) << 4) + 8u * (tq & 1);
+                    const uint2 lo = lds64_ring(box + row_lo + off);
+                    const uint2 hi = lds64_ring(box + row_hi + off);
+                    // B: x[token][kk + 16 tq, +16) of tokens 8 mb + g
+                    uint32_t xb[MB][8];
 #pragma unroll
-                    for (int gm = 0; gm < 4; ++gm) {
-                        const int kk = kb + 256 * h + 64 * gm;  // first k of the group
-                        if (kk >= kend) break;
-                        // 8 code bytes of the group for each row: 16-byte chunk
-                        // 2 gm + tq / 2 of the row, swizzled by the row (rho < 8)
-                        const uint32_t off =
-                            (static_cast<uint32_t>((2 * gm + (tq >> 1)) ^ rho) << 4) + 8u * (tq & 1);
-                        const uint2 lo = lds64_ring(box + row_lo + off);
-                        const uint2 hi = lds64_ring(box + row_hi + off);
-                        // B: x[token][kk + 16 tq, +16) of tokens 8 mb + g
-                        uint32_t xb[MB][8];
+                    for (int mb = 0; mb < MB; ++mb) {
+                        const int tok = 8 * mb + g;
+                        if (tok < p.M) {
+                            const uint32_t a = xlane + tok * p.x_pitch + 2u * (kk - k0);
+                            const uint4 v0 = lds128(a), v1 = lds128(a + 16);
+                            xb[mb][0] = v0.x; xb[mb][1] = v0.y; xb[mb][2] = v0.z; xb[mb][3] = v0.w;
+                            xb[mb][4] = v1.x; xb[mb][5] = v1.y; xb[mb][6] = v1.z; xb[mb][7] = v1.w;
+                        } else {
 #pragma unroll
-                        for (int mb = 0; mb < MB; ++mb) {
-                            const int tok = 8 * mb + g;
-                            if (tok < p.M) {
-                                const uint32_t a = xlane + tok * p.x_pitch + 2u * (kk - k0);
-                                const uint4 v0 = lds128(a), v1 = lds128(a + 16);
-                                xb[mb][0] = v0.x; xb[mb][1] = v0.y; xb[mb][2] = v0.z; xb[mb][3] = v0.w;
-                                xb[mb][4] = v1.x; xb[mb][5] = v1.y; xb[mb][6] = v1.z; xb[mb][7] = v1.w;
-                            } else {
-#pragma unroll
-                                for (int q = 0; q < 8; ++q) xb[mb][q] = 0u;
-                            }
+                            for (int q = 0; q < 8; ++q) xb[mb][q] = 0u;
                         }
-                        float d[MB][4];
+                    }
+                    float d[MB][4];
+#pragma unroll
+                    for (int mb = 0; mb < MB; ++mb)
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) d[mb][q] = 0.f;
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const uint32_t wl = (t < 2) ? lo.x : lo.y;
+                        const uint32_t wh = (t < 2) ? hi.x : hi.y;
+                        uint32_t a[4];
+                        if (t & 1) {
+                            a[0] = lut<2>(wl, lane4);
+                            a[1] = lut<2>(wh, lane4);
+                            a[2] = lut<3>(wl, lane4);
+                            a[3] = lut<3>(wh, lane4);
+                        } else {
+                            a[0] = lut<0>(wl, lane4);
+                            a[1] = lut<0>(wh, lane4);
+                            a[2] = lut<1>(wl, lane4);
+                            a[3] = lut<1>(wh, lane4);
+                        }
 #pragma unroll
                         for (int mb = 0; mb < MB; ++mb)
+                            mma_16816(d[mb], a, xb[mb][2 * t], xb[mb][2 * t + 1], d[mb]);
+                    }
+                    const float s1 = (j & 1) ? half_hi(sc_lo[j >> 1]) : half_lo(sc_lo[j >> 1]);
+                    const float s2 = (j & 1) ? half_hi(sc_hi[j >> 1]) : half_lo(sc_hi[j >> 1]);
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) d[mb][q] = 0.f;
+                    for (int mb = 0; mb < MB; ++mb) {
+                        acc[mb][0] = fmaf(s1, d[mb][0], acc[mb][0]);
+                        acc[mb][1] = fmaf(s1, d[mb][1], acc[mb][1]);
+                        acc[mb][2] = fmaf(s2, d[mb][2], acc[mb][2]);
+                        acc[mb][3] = fmaf(s2, d[mb][3], acc[mb][3]);
+                    }
+                };
+                if (kb + kStageK <= kend) {
+                    // a full stage: no branch between the groups
 #pragma unroll
-                        for (int t = 0; t < 4; ++t) {
-                            const uint32_t wl = (t < 2) ? lo.x : lo.y;
-                            const uint32_t wh = (t < 2) ? hi.x : hi.y;
-                            uint32_t a[4];
-                            if (t & 1) {
-                                a[0] = lut<2>(wl, lane4);
-                                a[1] = lut<2>(wh, lane4);
-                                a[2] = lut<3>(wl, lane4);
-                                a[3] = lut<3>(wh, lane4);
-                            } else {
-                                a[0] = lut<0>(wl, lane4);
-                                a[1] = lut<0>(wh, lane4);
-                                a[2] = lut<1>(wl, lane4);
-                                a[3] = lut<1>(wh, lane4);
-                            }
+                    for (int j = 0; j < 8; ++j) group(j);
+                } else {
 #pragma unroll
-                            for (int mb = 0; mb < MB; ++mb)
-                                mma_16816(d[mb], a, xb[mb][2 * t], xb[mb][2 * t + 1], d[mb]);
-                        }
-                        const int j = 4 * h + gm;  // group of the stage
-                        const float s1 = (j & 1) ? half_hi(sc_lo[j >> 1]) : half_lo(sc_lo[j >> 1]);
-                        const float s2 = (j & 1) ? half_hi(sc_hi[j >> 1]) : half_lo(sc_hi[j >> 1]);
-#pragma unroll
-                        for (int mb = 0; mb < MB; ++mb) {
-                            acc[mb][0] = fmaf(s1, d[mb][0], acc[mb][0]);
-                            acc[mb][1] = fmaf(s1, d[mb][1], acc[mb][1]);
-                            acc[mb][2] = fmaf(s2, d[mb][2], acc[mb][2]);
-                            acc[mb][3] = fmaf(s2, d[mb][3], acc[mb][3]);
-                        }
+                    for (int j = 0; j < 8; ++j) {
+                        if (kb + 64 * j >= kend) break;
+                        group(j);
                     }
                 }
             }
