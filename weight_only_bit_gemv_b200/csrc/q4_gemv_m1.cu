@@ -366,10 +366,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
         srow_lo = p.scales + static_cast<int64_t>(r0 + min(16 * st + g, nrows - 1)) * p.G;
         srow_hi = p.scales + static_cast<int64_t>(r0 + min(16 * st + g + 8, nrows - 1)) * p.G;
     };
+    int soff[kUPW];  // whole rows: the span of unit j never changes
+#pragma unroll
+    for (int j = 0; j < kUPW; ++j) soff[j] = min(2 * (warp + kCW * j) + (tq & 1), p.S - 1);
     auto next_scales = [&](uint32_t (&out)[kUPW][2]) {
 #pragma unroll
         for (int j = 0; j < kUPW; ++j) out[j][0] = out[j][1] = 0u;
-        if (sleft > 0) {
+        if (kWhole) {
+            if (sleft > 0) {
+#pragma unroll
+                for (int j = 0; j < kUPW; ++j) {
+                    out[j][0] = load_scales<kEvenG>(p, srow_lo, soff[j]);
+                    out[j][1] = load_scales<kEvenG>(p, srow_hi, soff[j]);
+                }
+                --sleft;
+                ++st;
+                scale_rows();
+            }
+        } else if (sleft > 0) {
 #pragma unroll
             for (int j = 0; j < kUPW; ++j) {
                 const int sp = min(2 * (scc * upk + warp + kCW * j) + (tq & 1), p.S - 1);
@@ -534,12 +548,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
         }
         for (int t = pt0; t < pt1; ++t) {
             float acc_lo = 0.f, acc_hi = 0.f;
-            for (int c = 0; c < p.C; ++c) {
+            for (int c = 0; c < (kWhole ? 1 : p.C); ++c) {
                 if (!bad && !mbar_wait(bars + 8u * slot, fparity)) {
                     bad = true;
                     if (lane == 0) atomicOr(&g_gemv_m1_error, 0x800u);
                 }
-                const int units = (min(p.KC, p.rowbytes - c * p.KC) + 127) >> 7;
+                const int units = kWhole ? upk : (min(p.KC, p.rowbytes - c * p.KC) + 127) >> 7;
                 const uint32_t a0 = ring_lane + slot * p.stage_bytes + 128 * warp;
 #pragma unroll
                 for (int j = 0; j < kUPW; ++j) {
