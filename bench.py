@@ -57,8 +57,8 @@ def peaks():
 # (4096 -> 22016) from an ncu capture, with the SHA-1 of the kernel source it
 # was taken on; when the source changes the figure no longer applies and the
 # bench reports null.
-GEMV_TRAFFIC = {"bytes": 47959296 + 4608,
-                "source_sha1": "966a54e51fcdce0c248501b0321ccd7c4e6a4842",
+GEMV_TRAFFIC = {"bytes": 47952640 + 768,
+                "source_sha1": "70830b055b063c710589e5a1ee77f560a7d94dda",
                 "capture": "ncu --set full --clock-control none -k regex:gemv_m1 -s 2 -c 1 "
                            "python -m weight_only_bit_gemv_b200.profile_case --M 1 --iters 5 "
                            "--copies 2 --workload llama2_7b_layer --linear gate_up"}
