@@ -136,8 +136,9 @@ q4_status q4_gemv(const uint8_t* codes, const uint16_t* scales,
  * Source: "deep-fold", "Method" table (prompt processing: a tensor-core NF4
  * GEMM that rebuilds weights into fragments); "Trapetum" overview, "What it
  * does" (speculative decoding verifies a few drafted tokens at once).
- * M <= 16 (verify batches) runs the same kernel family as q4_gemv, exact
- * products with binary32 accumulation.  M > 16 (prefill chunks) runs a tcgen05
+ * M <= 16 (verify batches) rebuilds binary16 codebook values once per weight
+ * for all M tokens (mma.sync, tokens as columns): exact products with binary32
+ * accumulation, each group's sum scaled in binary32, as q4_gemv.  M > 16 (prefill chunks) runs a tcgen05
  * tensor-core kernel: each weight is rebuilt as binary16(codebook * scale),
  * x is rounded to binary16, and products accumulate in binary32 in tensor
  * memory.  Either way the result is within 1e-4 * sum_k |W x| + 1e-6 of the
