@@ -54,6 +54,7 @@ constexpr uint32_t kRingOff = kLutBytes;
 constexpr uint32_t kBarOff = kRingOff + kNS * kStageBytes;
 constexpr uint32_t kXOff = kBarOff + 128;
 constexpr int kMaxSplits = 16;
+constexpr int kXRounds = 8;                    // x chunks in flight per thread in the set-up
 
 struct SmallP {
     const uint16_t* scales;
@@ -214,20 +215,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(smem + tid * 256 + 16 * ((i + lane) & 7)) =
                 make_uint4(ent, ent, ent, ent);
         // x[m][k0, k0 + KR) as binary16, zeros past K
+        // (all loads of a batch are issued before the first store: one
+        // memory latency per batch of kXRounds chunks per thread)
         const int chunks = p.KR / 8;
-        for (int i = tid; i < p.M * chunks; i += kCW * 32) {
-            const int m = i / chunks, j = i - m * chunks;
-            const int k = k0 + 8 * j;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (k < p.K) {
-                const uint4 b = __ldg(reinterpret_cast<const uint4*>(
-                    p.x + static_cast<int64_t>(m) * p.K + k));
-                v.x = cvt_bf16x2_f16x2(b.x);
-                v.y = cvt_bf16x2_f16x2(b.y);
-                v.z = cvt_bf16x2_f16x2(b.z);
-                v.w = cvt_bf16x2_f16x2(b.w);
+        const int total = p.M * chunks;
+        for (int i0 = 0; i0 < total; i0 += kXRounds * kCW * 32) {
+            uint4 b[kXRounds];
+#pragma unroll
+            for (int r = 0; r < kXRounds; ++r) {
+                const int i = i0 + tid + r * kCW * 32;
+                const int m = i / chunks, j = i - m * chunks;
+                const int k = k0 + 8 * j;
+                b[r] = make_uint4(0u, 0u, 0u, 0u);
+                if (i < total && k < p.K)
+                    b[r] = __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * p.K + k));
             }
-            *reinterpret_cast<uint4*>(smem + kXOff + m * p.x_pitch + 16 * j) = v;
+#pragma unroll
+            for (int r = 0; r < kXRounds; ++r) {
+                const int i = i0 + tid + r * kCW * 32;
+                if (i < total) {
+                    const int m = i / chunks, j = i - m * chunks;
+                    uint4 v;
+                    v.x = cvt_bf16x2_f16x2(b[r].x);
+                    v.y = cvt_bf16x2_f16x2(b[r].y);
+                    v.z = cvt_bf16x2_f16x2(b[r].z);
+                    v.w = cvt_bf16x2_f16x2(b[r].w);
+                    *reinterpret_cast<uint4*>(smem + kXOff + m * p.x_pitch + 16 * j) = v;
+                }
+            }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
     }
