@@ -206,6 +206,7 @@ def test_tiny_config_gemv():
     (1, 1, 64), (1, 7, 128), (1, 17, 448), (1, 1000, 4160), (1, 33, 28672),
     (3, 100, 192), (8, 129, 1024), (9, 31, 2048), (16, 300, 4096), (16, 64, 14336),
     (2, 4096, 11008), (5, 257, 4160), (12, 1000, 2112), (7, 129, 320), (11, 2, 64),
+    (13, 1, 64), (16, 129, 16448), (6, 4100, 2560), (10, 640, 7168),
     (17, 130, 512), (64, 257, 1088), (100, 96, 4096),
     (300, 200, 640), (257, 130, 2048), (48, 1000, 4160)])
 def test_ragged_shapes(M, N, K):
