@@ -39,9 +39,10 @@
 //    kernel; otherwise x goes to shared memory in that column layout (for
 //    K <= 8192 inside the unused half of the table rows).  Scales are read
 //    from global memory by the consumers, stages ahead.
-//  * The warps of a CTA add their tile sums into a shared-memory row
-//    accumulator; the CTA writes each y element once (no split-K between
-//    CTAs, no zeroing of y, no global atomics).
+//  * Each warp stores its tile sums in its own shared-memory slot (no
+//    atomics); at the end of a pass of tiles the CTA adds the warps' slots
+//    and writes each y element once (no split-K between CTAs, no zeroing of
+//    y, no global atomics).
 //  * Programmatic dependent launch: the kernel lets the next kernel on the
 //    stream launch at once, prefetches the first stages of its weights into
 //    L2 (a prefetch only warms the cache, so it never reads stale data), and
@@ -62,14 +63,15 @@ constexpr int kBase = 1024;               // shared-window address of dynamic sh
 constexpr int kLutBytes = 65536;          // 256 rows of 256 bytes; lane copies in the first 128
 constexpr int kSpan = 128;                // k per span (64 code bytes)
 constexpr int kMaxKC = 2048;              // code bytes of a row per stage
-constexpr int kPassTiles = 128;           // tiles per pass of the shared row accumulator
+constexpr int kMinPassTiles = 16;         // tiles per pass of the per-warp row partials (at least)
+constexpr int kMaxPassTiles = 64;
+constexpr uint32_t kTileSlotBytes = kCW * 16 * 4;  // one tile's partials of every warp
 constexpr int kAhead = 3;                 // scale prefetch distance, in stages
 constexpr int kMaxStages = 6;
 constexpr int kXEmbedSpans = 64;          // spans whose x fits in the table rows' free halves
 constexpr int kXRounds = 13;              // x chunk loads per consumer thread: K <= 13 * 256 * 8
 constexpr uint32_t kAccOff = kLutBytes;
-constexpr uint32_t kBarOff = kAccOff + kPassTiles * 16 * 4;
-constexpr uint32_t kXOff = kBarOff + 128;
+
 static_assert(2 * kMaxStages * 8 <= 128, "barriers overflow their area");
 
 struct M1 {
@@ -84,6 +86,8 @@ struct M1 {
     int KC;          // code bytes of a row per stage (the ring's row pitch)
     int C;           // stages per 16-row tile
     int NS;          // ring stages
+    int PT;          // tiles per pass of the row partials
+    uint32_t bar_off, x_off;  // barriers (128 bytes), then x when it is not in the table rows
     uint32_t ring_off, stage_bytes;
 };
 
@@ -230,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
         if (tid == 0) atomicOr(&g_gemv_m1_error, 0x100u);
         return;
     }
-    const uint32_t bars = base + kBarOff;
+    const uint32_t bars = base + p.bar_off;
     const int NS = p.NS;
     const int r0 = static_cast<int>(static_cast<int64_t>(p.N) * blockIdx.x / gridDim.x);
     const int r1 = static_cast<int>(static_cast<int64_t>(p.N) * (blockIdx.x + 1) / gridDim.x);
@@ -462,7 +466,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
             // of that group), else zeros; chunks past K are zeros.
             auto chunk_off = [&](int s, int q, int par, int j) -> uint32_t {
                 return kXEmb ? (4 * s + q) * 256 + 128 + par * 64 + j * 16
-                             : kXOff + s * 512 + q * 128 + par * 64 + j * 16;
+                             : p.x_off + s * 512 + q * 128 + par * 64 + j * 16;
             };
 #pragma unroll
             for (int i = 0; i < kXRounds; ++i) {
@@ -535,14 +539,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
     uint32_t xlane = 0;
     int slot = 0;
     uint32_t fparity = 0;
-    for (int pt0 = 0; pt0 < T; pt0 += kPassTiles) {
-        const int pt1 = min(T, pt0 + kPassTiles);
-        for (int i = tid; i < kPassTiles * 16; i += kCW * 32) acc_s[i] = 0.f;
-        asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
+    for (int pt0 = 0; pt0 < T; pt0 += p.PT) {
+        const int pt1 = min(T, pt0 + p.PT);
         if (!started) {
+            asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
             // formed after the first consumer barrier: the empty asm keeps every
             // x read below it
-            xlane = base + (kXEmb ? 128u : kXOff) + ((g >> 1) & 1) * kXSpan + (g & 1) * 64 + tq * 16;
+            xlane = base + (kXEmb ? 128u : p.x_off) + ((g >> 1) & 1) * kXSpan + (g & 1) * 64 + tq * 16;
             asm volatile("" : "+r"(xlane)::"memory");
             started = true;
         }
@@ -587,14 +590,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
             acc_lo += __shfl_xor_sync(0xFFFFFFFFu, acc_lo, 1);
             acc_hi += __shfl_xor_sync(0xFFFFFFFFu, acc_hi, 1);
             if (tq == 0) {
-                const int rl = 16 * (t - pt0) + g;
-                if (16 * t + g < nrows) atomicAdd(acc_s + rl, acc_lo);
-                if (16 * t + g + 8 < nrows) atomicAdd(acc_s + rl + 8, acc_hi);
+                // this warp's partials of the tile's rows: slot [tile][warp][row]
+                float* slot_w = acc_s + ((t - pt0) * kCW + warp) * 16;
+                slot_w[g] = acc_lo;
+                slot_w[g + 8] = acc_hi;
             }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
         const int row_end = min(nrows, 16 * pt1);
-        for (int r = 16 * pt0 + tid; r < row_end; r += kCW * 32) p.y[r0 + r] = acc_s[r - 16 * pt0];
+        for (int r = 16 * pt0 + tid; r < row_end; r += kCW * 32) {
+            const int rl = r - 16 * pt0;
+            const float* q = acc_s + (rl >> 4) * (kCW * 16) + (rl & 15);
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < kCW; ++w) sum += q[16 * w];
+            p.y[r0 + r] = sum;
+        }
         asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
     }
 }
@@ -656,14 +667,28 @@ cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const u
     }
     if (p.K > kXRounds * kCW * 32 * 8) return cudaErrorNotSupported;
     const bool xemb = p.SP <= kXEmbedSpans;
-    const uint32_t x_end = xemb ? kXOff : kXOff + static_cast<uint32_t>(p.SP) * 512u;
-    p.ring_off = (x_end + 127u) & ~127u;
     p.stage_bytes = static_cast<uint32_t>(16 * p.KC);
-    const int room = dev.smem_optin - static_cast<int>(p.ring_off) - 128;  // 128: read slack
-    int ns = room / static_cast<int>(p.stage_bytes);
+    // Shared memory: table | row partials (PT tiles) | barriers | x (when not
+    // in the table rows) | ring.  The ring's stage count is set with the
+    // smallest partials area; the partials then take what the ring leaves,
+    // up to kMaxPassTiles tiles (fewer passes, fewer barriers).
+    auto layout = [&](int pt) {
+        p.PT = pt;
+        p.bar_off = kAccOff + static_cast<uint32_t>(pt) * kTileSlotBytes;
+        p.x_off = p.bar_off + 128u;
+        const uint32_t x_end = xemb ? p.x_off : p.x_off + static_cast<uint32_t>(p.SP) * 512u;
+        p.ring_off = (x_end + 127u) & ~127u;
+        return dev.smem_optin - static_cast<int>(p.ring_off) - 128;  // 128: read slack
+    };
+    int ns = layout(kMinPassTiles) / static_cast<int>(p.stage_bytes);
     if (ns > kMaxStages) ns = kMaxStages;
     if (ns < 2) return cudaErrorNotSupported;
     p.NS = ns;
+    const int64_t tiles_per_cta = ((N + dev.sm_count - 1) / dev.sm_count + 15) / 16 + 1;
+    const int pt_cap = static_cast<int>(tiles_per_cta < kMaxPassTiles ? tiles_per_cta : kMaxPassTiles);
+    for (int pt = pt_cap; pt > kMinPassTiles; --pt)
+        if (layout(pt) >= ns * static_cast<int>(p.stage_bytes)) break;
+    if (layout(p.PT) < ns * static_cast<int>(p.stage_bytes)) layout(kMinPassTiles);
     const int smem = static_cast<int>(p.ring_off + ns * p.stage_bytes) + 128;
 
     const int64_t tiles = (N + 15) / 16;
