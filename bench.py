@@ -14,7 +14,8 @@ The JSON line reports:
   roofline      the gate_up launch (largest share of the step), its algorithmic
                 bytes / its mean CUDA-event duration, against the measured HBM peak
   e2e           the same metric through the Python API per step, with x copied
-                from pinned host memory and y read back every step
+                from pinned host memory and y read back every step (the step's
+                calls replayed from a CUDA graph)
   cpu_baseline  the oracle (single-threaded C) on the same layer, on the host
   gemm_prefill  q4_gemm at M = 256 on the Llama-2-70B linears: TFLOP/s
 
@@ -57,8 +58,8 @@ def peaks():
 # (4096 -> 22016) from an ncu capture, with the SHA-1 of the kernel source it
 # was taken on; when the source changes the figure no longer applies and the
 # bench reports null.
-GEMV_TRAFFIC = {"bytes": 47952640 + 768,
-                "source_sha1": "70830b055b063c710589e5a1ee77f560a7d94dda",
+GEMV_TRAFFIC = {"bytes": 47954688 + 1024,
+                "source_sha1": "944c51b3f5a14d3400fd5705a72a5d4e68c84836",
                 "capture": "ncu --set full --clock-control none -k regex:gemv_m1 -s 2 -c 1 "
                            "python -m weight_only_bit_gemv_b200.profile_case --M 1 --iters 5 "
                            "--copies 2 --workload llama2_7b_layer --linear gate_up"}
@@ -297,19 +298,43 @@ def run_ours(args, world, rank, local):
     dom_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
 
     # ---- end to end through the Python API with host buffers -----------------
-    xh = [torch.empty((1, L["lin"].K), dtype=torch.bfloat16).pin_memory() for L in lins]
-    for h, L in zip(xh, lins):
-        h.copy_(L["x"].cpu())
-    yh = [torch.empty((1, L["lin"].N), dtype=torch.float32).pin_memory() for L in lins]
+    # The step's inputs (x of the four linears) sit in one pinned host buffer
+    # and its results (the four y) in one device buffer: every step copies x
+    # host -> device, runs the four q4_gemv calls and copies y device -> host.
+    # Each step is replayed from a CUDA graph captured over those API calls
+    # (one graph per weight copy).
+    xs_len = [L["lin"].K for L in lins]
+    ys_len = [L["lin"].N for L in lins]
+    xh_all = torch.empty(sum(xs_len), dtype=torch.bfloat16).pin_memory()
+    yh_all = torch.empty(sum(ys_len), dtype=torch.float32).pin_memory()
+    xd_all = torch.empty(sum(xs_len), dtype=torch.bfloat16, device=dev)
+    yd_all = torch.empty(sum(ys_len), dtype=torch.float32, device=dev)
+    xh_all.copy_(torch.cat([L["x"].reshape(-1).cpu() for L in lins]))
+    xd_views = [v.view(1, -1) for v in torch.split(xd_all, xs_len)]
+    yd_views = [v.view(1, -1) for v in torch.split(yd_all, ys_len)]
+    h2d = xh_all.numel() * 2
+    d2h = yh_all.numel() * 4
     e2e_steps = min(K, 2000)
-    h2d = sum(h.numel() * 2 for h in xh)
-    d2h = sum(h.numel() * 4 for h in yh)
+
+    def e2e_step(c):
+        xd_all.copy_(xh_all, non_blocking=True)
+        for j, L in enumerate(lins):
+            q4.q4_gemv(L["copies"][c][0], L["copies"][c][1], cb, xd_views[j], yd_views[j])
+        yh_all.copy_(yd_all, non_blocking=True)
+
     with torch.cuda.stream(stream):
-        for i in range(min(W, 20) + 1):
-            for j, L in enumerate(lins):
-                L["x"].copy_(xh[j], non_blocking=True)
-                q4.q4_gemv(L["copies"][0][0], L["copies"][0][1], cb, L["x"], L["y"])
-                yh[j].copy_(L["y"], non_blocking=True)
+        for c in range(COPIES):
+            e2e_step(c)  # eager once per copy (first-call set-up outside the graph)
+    stream.synchronize()
+    g_e2e = []
+    for c in range(COPIES):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            e2e_step(c)
+        g_e2e.append(g)
+    with torch.cuda.stream(stream):
+        for i in range(max(W, 3) * COPIES):
+            g_e2e[i % COPIES].replay()
     stream.synchronize()
     barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
@@ -317,15 +342,14 @@ def run_ours(args, world, rank, local):
     with torch.cuda.stream(stream):
         e0.record()
         for i in range(e2e_steps):
-            c = i % COPIES
-            for j, L in enumerate(lins):
-                L["x"].copy_(xh[j], non_blocking=True)
-                q4.q4_gemv(L["copies"][c][0], L["copies"][c][1], cb, L["x"], L["y"])
-                yh[j].copy_(L["y"], non_blocking=True)
+            g_e2e[i % COPIES].replay()
         e1.record()
     e1.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    # the last step's y arrived on the host: it must equal the device-timed y
+    e2e_match = bool(torch.equal(yh_all, torch.cat([L["y"].reshape(-1).cpu() for L in lins])))
+    del g_e2e
 
     # ---- prefill q4_gemm, M = 256, Llama-2-70B linears --------------------------
     gemm = None
@@ -385,7 +409,10 @@ def run_ours(args, world, rank, local):
             "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
             "ms_per_step": round(e2e_ms, 6),
-            "api": "weight_only_bit_gemv_b200.q4_gemv per linear, eager, host x in / host y out",
+            "y_matches_device_path": e2e_match,
+            "api": "weight_only_bit_gemv_b200.q4_gemv per linear; per step one pinned host-to-device "
+                   "copy of the four x and one device-to-host copy of the four y, the step's API "
+                   "calls captured in a CUDA graph",
         },
         "gpu_launches": 4 * K,
         "clocks": clk,
