@@ -354,7 +354,7 @@ def run_ours(args, world, rank, local):
     # ---- prefill q4_gemm, M = 256, Llama-2-70B linears --------------------------
     gemm = None
     if not args.no_gemm:
-        gemm = bench_prefill(dev, cb, stream, tc_peak, M=256)
+        gemm = bench_prefill(dev, cb, stream, tc_peak, hbm_peak)
 
     # ---- other workloads: a full 8B decode step, small-M verify batches --------
     step8b = None if args.no_step else bench_decode_step(dev, cb, stream, hbm_peak)
@@ -429,54 +429,77 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def bench_prefill(dev, cb, stream, tc_peak, M=256):
+def bench_prefill(dev, cb, stream, tc_peak, hbm_peak, Ms=(32, 128, 256, 512), main_M=256):
+    """q4_gemm on the Llama-2-70B linears at each M of ``Ms``: each linear is
+    packed once and timed from a CUDA graph of 4 back-to-back calls."""
     import torch
     import weight_only_bit_gemv_b200 as q4
     wl = synth.WORKLOADS["llama2_70b_prefill"]
-    out = {}
-    total_flop, total_ms = 0.0, 0.0
+    per_m = {M: {"flop": 0.0, "bytes": 0.0, "ms": 0.0, "roof_ms": 0.0, "lin": {}} for M in Ms}
     for lin in wl.linears:
         seed = synth.seed_for(wl.index, 0, lin.name)
         w = synth.weights_device(seed, lin.N, lin.K, wl.w_std, dev)
         codes, scales = q4.q4_pack(w, cb)
         del w
-        x = synth.activations_device(synth.x_seed(seed) + M, M, lin.K, dev)
-        y = torch.empty((M, lin.N), dtype=torch.float32, device=dev)
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                q4.q4_gemm(codes, scales, cb, x, y)
-            stream.synchronize()
-            # a CUDA graph of `per` calls: the device time of the calls, without
-            # the host's per-call work (tensor-map encoding, argument checks)
-            per = 4
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for _ in range(per):
+        for M in Ms:
+            x = synth.activations_device(synth.x_seed(seed) + M, M, lin.K, dev)
+            y = torch.empty((M, lin.N), dtype=torch.float32, device=dev)
+            with torch.cuda.stream(stream):
+                for _ in range(3):
                     q4.q4_gemm(codes, scales, cb, x, y)
-            g.replay()
-            stream.synchronize()
-            reps = 5
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record()
-            for _ in range(reps):
+                stream.synchronize()
+                # a CUDA graph of `per` calls: the device time of the calls,
+                # without the host's per-call work (tensor-map encoding, checks)
+                per = 4
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    for _ in range(per):
+                        q4.q4_gemm(codes, scales, cb, x, y)
                 g.replay()
-            e1.record()
-        e1.synchronize()
-        ms = e0.elapsed_time(e1) / (reps * per)
-        del g
-        flop = 2.0 * M * lin.N * lin.K
-        out[lin.name] = {"us": round(ms * 1e3, 2), "tflops": round(flop / (ms * 1e-3) / 1e12, 2)}
-        total_flop += flop
-        total_ms += ms
-        del codes, scales, x, y
+                stream.synchronize()
+                reps = 5
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(reps):
+                    g.replay()
+                e1.record()
+            e1.synchronize()
+            ms = e0.elapsed_time(e1) / (reps * per)
+            del g
+            flop = 2.0 * M * lin.N * lin.K
+            nbytes = algo_bytes(M, lin.N, lin.K)
+            r = per_m[M]
+            r["lin"][lin.name] = {"us": round(ms * 1e3, 2), "tflops": round(flop / (ms * 1e-3) / 1e12, 2)}
+            r["flop"] += flop
+            r["bytes"] += nbytes
+            r["ms"] += ms
+            # roofline time of this linear: the slower of its flops at the
+            # tensor peak and its bytes at the HBM peak
+            r["roof_ms"] += max(flop / (tc_peak * 1e12), nbytes / (hbm_peak * 1e9)) * 1e3
+            del x, y
+        del codes, scales
         torch.cuda.empty_cache()
-    tf = total_flop / (total_ms * 1e-3) / 1e12
-    return {"workload": "llama2_70b_prefill layer (4 linears), M=256", "tflops": round(tf, 2),
-            "frac_of_bf16_peak": round(tf / tc_peak, 4), "per_linear": out,
-            "timing": "CUDA graph of 4 back-to-back q4_gemm calls (x conversion, y zeroing when K "
-                      "is split, and the tensor-core GEMM), replayed 5 times",
-            "note": "no L2 flush: each linear is 37-253 MB of packed weights, read once per launch"}
+    sweep = {}
+    for M in Ms:
+        r = per_m[M]
+        tf = r["flop"] / (r["ms"] * 1e-3) / 1e12
+        gbs = r["bytes"] / (r["ms"] * 1e-3) / 1e9
+        hbm_bound = r["bytes"] / (hbm_peak * 1e9) > r["flop"] / (tc_peak * 1e12)
+        sweep[f"M={M}"] = {"tflops": round(tf, 2), "gbs": round(gbs, 1),
+                           "bound": "hbm" if hbm_bound else "tensor",
+                           "frac_of_roofline": round(r["roof_ms"] / r["ms"], 4),
+                           "us": round(r["ms"] * 1e3, 2)}
+    m = per_m[main_M]
+    tf = m["flop"] / (m["ms"] * 1e-3) / 1e12
+    return {"workload": f"llama2_70b_prefill layer (4 linears), M={main_M}", "tflops": round(tf, 2),
+            "frac_of_bf16_peak": round(tf / tc_peak, 4), "per_linear": m["lin"],
+            "sweep": sweep,
+            "timing": "per linear and M: CUDA graph of 4 back-to-back q4_gemm calls (x conversion, "
+                      "y zeroing when K is split, and the tensor-core GEMM), replayed 5 times",
+            "note": "no L2 flush: each linear is 37-253 MB of packed weights, read once per launch; "
+                    "frac_of_roofline = sum over the linears of max(flop / tensor peak, bytes / HBM "
+                    "peak) over the measured time"}
 
 
 def bench_decode_step(dev, cb, stream, hbm_peak, reps=20):

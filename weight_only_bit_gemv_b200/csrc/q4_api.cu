@@ -171,6 +171,14 @@ q4_status q4_gemm(const uint8_t* codes, const uint16_t* scales, const uint16_t* 
     if (M <= 16)
         return after_launch(
             launch_small_m(codes, scales, codebook, x, y, static_cast<int>(M), N, K, stream, dev));
+    if (M <= 32) {
+        // still weight-streaming: the CUDA-core decode kernel beats the
+        // tensor-core pipeline here (its per-group MMA issue does not shrink with M)
+        cudaError_t e = launch_gemm_small(codes, scales, codebook, x, y, static_cast<int>(M), N, K,
+                                          stream, dev);
+        if (e != cudaErrorNotSupported) return after_launch(e);
+        (void)cudaGetLastError();
+    }
     return after_launch(launch_prefill(codes, scales, codebook, x, y, M, N, K, stream, dev));
 }
 
@@ -188,6 +196,12 @@ q4_status q4_gemm_noalloc(const uint8_t* codes, const uint16_t* scales, const ui
     if (M <= 16)
         return after_launch(
             launch_small_m(codes, scales, codebook, x, y, static_cast<int>(M), N, K, stream, dev));
+    if (M <= 32) {
+        cudaError_t e = launch_gemm_small(codes, scales, codebook, x, y, static_cast<int>(M), N, K,
+                                          stream, dev);
+        if (e != cudaErrorNotSupported) return after_launch(e);
+        (void)cudaGetLastError();
+    }
     return after_launch(launch_prefill_noalloc(codes, scales, codebook, x, y, M, N, K, stream, dev));
 }
 

@@ -1,4 +1,5 @@
-// q4_gemm_small.cu -- q4_gemm for M = 2..16 tokens (verify batches) on sm_100a.
+// q4_gemm_small.cu -- q4_gemm for M = 2..32 tokens (verify batches, short
+// prefill chunks) on sm_100a.
 //
 // What it computes: y[m][n] = sum_g scale[n][g] * sum_{k in g} cb[code(n,k)] * x[m][k]
 // ("deep-fold", "Method": 64-weight groups, four-bit codes, one FP16 scale,
@@ -6,8 +7,8 @@
 // few drafted tokens of speculative decoding are checked in one pass), with
 // exact binary16 products and fp32 sums, as the M = 1 kernel.
 //
-// Why this shape.  Up to 16 tokens the work is still a weight stream (under
-// 60 flop per byte), so the kernel is organised around reading each weight
+// Why this shape.  Up to 32 tokens the work is still a weight stream (under
+// 120 flop per byte), so the kernel is organised around reading each weight
 // once at HBM speed and decoding it once for all tokens.
 //  * A CTA takes blocks of 128 weight rows over one range of K.  Each of its
 //    8 consumer warps owns 16 of the rows for the whole range, so a row's
@@ -20,7 +21,7 @@
 //    per lane in shared memory (entry b of lane l at 256 b + 4 l), so one
 //    PRMT forms the address and one LDS returns two rebuilt weights.
 //  * The rebuilt weights are the A operand of mma.sync m16n8k16 and the
-//    tokens are the columns of B (8 per MMA; a second MMA for tokens 8-15).
+//    tokens are the columns of B (8 per MMA, one MMA per 8 tokens).
 //    Lane (g, tq) reads 8 code bytes of one group of its two rows, so the
 //    four k-steps of a group form one MMA chain: the group's fp32 partial sum
 //    is scaled by the group's own scale in fp32.
@@ -53,7 +54,7 @@ constexpr int kNS = 3;                         // ring stages
 constexpr uint32_t kRingOff = kLutBytes;
 constexpr uint32_t kBarOff = kRingOff + kNS * kStageBytes;
 constexpr uint32_t kXOff = kBarOff + 128;
-constexpr int kMaxSplits = 16;
+constexpr int kMaxSplits = 64;
 constexpr int kXRounds = 8;                    // x chunks in flight per thread in the set-up
 
 struct SmallP {
@@ -416,7 +417,7 @@ cudaError_t take_gemm_small_error(unsigned int* out) {
 cudaError_t launch_gemm_small(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                               const uint16_t* x, float* y, int M, int64_t N, int64_t K,
                               cudaStream_t s, const DeviceInfo& dev) {
-    if (M < 2 || M > 16 || dev.smem_reserved != kBase) return cudaErrorNotSupported;
+    if (M < 2 || M > 32 || dev.smem_reserved != kBase) return cudaErrorNotSupported;
     SmallP p{};
     p.scales = scales;
     p.cb = cb;
@@ -474,8 +475,14 @@ cudaError_t launch_gemm_small(const uint8_t* codes, const uint16_t* scales, cons
     if (M <= 8)
         return even ? launch_variant<1, true>(cmap, p, best_grid, smem, 40, s, dev)
                     : launch_variant<1, false>(cmap, p, best_grid, smem, 41, s, dev);
-    return even ? launch_variant<2, true>(cmap, p, best_grid, smem, 42, s, dev)
-                : launch_variant<2, false>(cmap, p, best_grid, smem, 43, s, dev);
+    if (M <= 16)
+        return even ? launch_variant<2, true>(cmap, p, best_grid, smem, 42, s, dev)
+                    : launch_variant<2, false>(cmap, p, best_grid, smem, 43, s, dev);
+    if (M <= 24)
+        return even ? launch_variant<3, true>(cmap, p, best_grid, smem, 44, s, dev)
+                    : launch_variant<3, false>(cmap, p, best_grid, smem, 45, s, dev);
+    return even ? launch_variant<4, true>(cmap, p, best_grid, smem, 46, s, dev)
+                : launch_variant<4, false>(cmap, p, best_grid, smem, 47, s, dev);
 }
 
 }  // namespace q4

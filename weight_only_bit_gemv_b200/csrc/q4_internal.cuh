@@ -47,7 +47,7 @@ cudaError_t launch_small_m(const uint8_t* codes, const uint16_t* scales, const u
 cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
                            const DeviceInfo& dev);
-// M in [2, 16]: TMA-fed row blocks, decoded weights on mma.sync with the
+// M in [2, 32]: TMA-fed row blocks, decoded weights on mma.sync with the
 // tokens as B columns, exact products.  Returns cudaErrorNotSupported when the
 // device's shared-memory layout or the shape does not fit it.
 cudaError_t launch_gemm_small(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
