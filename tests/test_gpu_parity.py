@@ -207,6 +207,7 @@ def test_tiny_config_gemv():
     (3, 100, 192), (8, 129, 1024), (9, 31, 2048), (16, 300, 4096), (16, 64, 14336),
     (2, 4096, 11008), (5, 257, 4160), (12, 1000, 2112), (7, 129, 320), (11, 2, 64),
     (13, 1, 64), (16, 129, 16448), (6, 4100, 2560), (10, 640, 7168),
+    (20, 4096, 4160), (32, 200, 24576), (25, 1, 64),
     (17, 130, 512), (64, 257, 1088), (100, 96, 4096),
     (300, 200, 640), (257, 130, 2048), (48, 1000, 4160)])
 def test_ragged_shapes(M, N, K):
