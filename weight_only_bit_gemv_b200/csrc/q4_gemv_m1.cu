@@ -65,7 +65,7 @@ constexpr int kSpan = 128;                // k per span (64 code bytes)
 constexpr int kMaxKC = 2048;              // code bytes of a row per stage
 constexpr int kMinPassTiles = 16;         // tiles per pass of the per-warp row partials (at least)
 constexpr int kMaxPassTiles = 64;
-constexpr uint32_t kTileSlotBytes = kCW * 16 * 4;  // one tile's partials of every warp
+constexpr uint32_t kTileSlotBytes = kCW * 16 * 4;  // one tile's partials of every warp, per token
 constexpr int kAhead = 3;                 // scale prefetch distance, in stages
 constexpr int kMaxStages = 6;
 constexpr int kXEmbedSpans = 64;          // spans whose x fits in the table rows' free halves
@@ -217,8 +217,9 @@ __device__ __forceinline__ uint32_t load_scales(const M1& p, const uint16_t* sro
     return ldg_u16(q) | (ldg_u16(q + (2 * s + 1 < p.G ? 1 : 0)) << 16);
 }
 
-template <bool kEvenG, bool kWhole, bool kXEmb>
+template <bool kEvenG, bool kWhole, bool kXEmb, int MT>
 __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
+    static_assert(MT == 1 || (MT == 2 && kWhole), "two tokens only with whole rows");
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, tq = lane & 3;
@@ -434,7 +435,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
             for (int j = 0; j < kUPW; ++j) {
                 const int U = warp + kCW * j;
                 const bool act = U < upk && (g & 1) == (tq >> 1);
-                const uint16_t* xs = p.x + kSpan * (2 * U + ((g >> 1) & 1)) + 32 * tq;
+                // two tokens: B columns 4-7 (lanes g >= 4) hold token 1
+                const uint16_t* xs = p.x + (MT == 2 ? (g >> 2) * p.K : 0) +
+                                     kSpan * (2 * U + ((g >> 1) & 1)) + 32 * tq;
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -586,12 +589,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
                     }
                 next_scales(sc[kAhead - 1]);
             }
-            // lanes tq = 0, 1 hold the two spans' sums of rows g, g + 8
+            // lanes tq = 0, 1 hold the two spans' sums of rows g, g + 8 for
+            // token 0; lanes tq = 2, 3 the same for token 1 (columns 4-7)
             acc_lo += __shfl_xor_sync(0xFFFFFFFFu, acc_lo, 1);
             acc_hi += __shfl_xor_sync(0xFFFFFFFFu, acc_hi, 1);
-            if (tq == 0) {
-                // this warp's partials of the tile's rows: slot [tile][warp][row]
-                float* slot_w = acc_s + ((t - pt0) * kCW + warp) * 16;
+            if (tq == 0 || (MT == 2 && tq == 2)) {
+                // this warp's partials of the tile's rows:
+                // slot [tile][warp][token][row]
+                float* slot_w = acc_s + (((t - pt0) * kCW + warp) * MT + (tq >> 1)) * 16;
                 slot_w[g] = acc_lo;
                 slot_w[g + 8] = acc_hi;
             }
@@ -600,20 +605,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
         const int row_end = min(nrows, 16 * pt1);
         for (int r = 16 * pt0 + tid; r < row_end; r += kCW * 32) {
             const int rl = r - 16 * pt0;
-            const float* q = acc_s + (rl >> 4) * (kCW * 16) + (rl & 15);
-            float sum = 0.f;
 #pragma unroll
-            for (int w = 0; w < kCW; ++w) sum += q[16 * w];
-            p.y[r0 + r] = sum;
+            for (int tok = 0; tok < MT; ++tok) {
+                const float* q = acc_s + ((rl >> 4) * kCW * MT + tok) * 16 + (rl & 15);
+                float sum = 0.f;
+#pragma unroll
+                for (int w = 0; w < kCW; ++w) sum += q[16 * MT * w];
+                p.y[static_cast<int64_t>(tok) * p.N + r0 + r] = sum;
+            }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
     }
 }
 
-template <bool kEvenG, bool kWhole, bool kXEmb>
+template <bool kEvenG, bool kWhole, bool kXEmb, int MT = 1>
 cudaError_t launch_variant(const M1& p, int grid, int smem, int slot, cudaStream_t s,
                            const DeviceInfo& dev) {
-    auto kern = gemv_m1_kernel<kEvenG, kWhole, kXEmb>;
+    auto kern = gemv_m1_kernel<kEvenG, kWhole, kXEmb, MT>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem, slot, dev.device);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -639,9 +647,9 @@ cudaError_t take_gemv_m1_error(unsigned int* out) {
 }
 
 cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
-                           const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
+                           const uint16_t* x, float* y, int M, int64_t N, int64_t K, cudaStream_t s,
                            const DeviceInfo& dev) {
-    if (dev.smem_reserved != kBase) return cudaErrorNotSupported;
+    if (dev.smem_reserved != kBase || M < 1 || M > 2) return cudaErrorNotSupported;
     M1 p{};
     p.codes = codes;
     p.scales = scales;
@@ -658,6 +666,7 @@ cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const u
     // multiple of 128 bytes travel whole (a tile is one contiguous copy);
     // longer rows in C segments of KC bytes (a multiple of 128).
     const bool whole = p.rowbytes <= kMaxKC && p.rowbytes % 128 == 0;
+    if (M == 2 && !whole) return cudaErrorNotSupported;  // two tokens: whole rows only
     if (whole) {
         p.C = 1;
         p.KC = p.rowbytes;
@@ -674,7 +683,7 @@ cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const u
     // up to kMaxPassTiles tiles (fewer passes, fewer barriers).
     auto layout = [&](int pt) {
         p.PT = pt;
-        p.bar_off = kAccOff + static_cast<uint32_t>(pt) * kTileSlotBytes;
+        p.bar_off = kAccOff + static_cast<uint32_t>(pt * M) * kTileSlotBytes;
         p.x_off = p.bar_off + 128u;
         const uint32_t x_end = xemb ? p.x_off : p.x_off + static_cast<uint32_t>(p.SP) * 512u;
         p.ring_off = (x_end + 127u) & ~127u;
@@ -694,6 +703,9 @@ cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const u
     const int64_t tiles = (N + 15) / 16;
     const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
     const bool even = (p.G & 1) == 0;
+    if (whole && M == 2)
+        return even ? launch_variant<true, true, true, 2>(p, grid, smem, 22, s, dev)
+                    : launch_variant<false, true, true, 2>(p, grid, smem, 23, s, dev);
     if (whole) {
         return even ? launch_variant<true, true, true>(p, grid, smem, 16, s, dev)
                     : launch_variant<false, true, true>(p, grid, smem, 17, s, dev);
