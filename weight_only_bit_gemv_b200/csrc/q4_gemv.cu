@@ -290,7 +290,7 @@ cudaError_t launch_variant(SmallM p, int slot, cudaStream_t s, const DeviceInfo&
 cudaError_t launch_small_m(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int M, int64_t N, int64_t K,
                            cudaStream_t s, const DeviceInfo& dev) {
-    if (M <= 2) {
+    if (M <= 4) {
         cudaError_t e = launch_gemv_m1(codes, scales, cb, x, y, M, N, K, s, dev);
         if (e != cudaErrorNotSupported) return e;
         (void)cudaGetLastError();

@@ -80,6 +80,7 @@ struct M1 {
     const uint16_t* cb;
     const uint16_t* x;
     float* y;
+    int M;           // tokens (1..4)
     int N, K, G, S;  // S = spans of 128 k (the last may hold one group)
     int SP;          // S rounded up to even: x holds a zero span S when S is odd
     int rowbytes;    // K / 2
@@ -178,11 +179,13 @@ __device__ __forceinline__ uint32_t lut(uint32_t word, uint32_t lane4) {
 
 __device__ __forceinline__ uint32_t lane4_of(int lane) { return static_cast<uint32_t>(lane) * 4u; }
 
-// One pass over the 128 k of this lane's row slots: eight MMAs in two
-// independent chains of four (the sums of k-steps 0-3 and 4-7), so that a
-// warp keeps more MMAs in flight.
-__device__ __forceinline__ void pass_mma(uint4 lo, uint4 hi, const uint32_t (&xr)[16],
-                                         uint32_t lane4, float (&d)[4], float (&e)[4]) {
+// One pass over the 128 k of this lane's row slots: eight MMAs per token
+// pair in two independent chains of four (the sums of k-steps 0-3 and 4-7),
+// so that a warp keeps more MMAs in flight; the rebuilt weights serve every
+// pair.
+template <int MP>
+__device__ __forceinline__ void pass_mma(uint4 lo, uint4 hi, const uint32_t (&xr)[MP][16],
+                                         uint32_t lane4, float (&d)[MP][4], float (&e)[MP][4]) {
     const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w};
     const uint32_t wh[4] = {hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
@@ -200,10 +203,13 @@ __device__ __forceinline__ void pass_mma(uint4 lo, uint4 hi, const uint32_t (&xr
             a[2] = lut<1>(l, lane4);
             a[3] = lut<1>(h, lane4);
         }
-        if (t < 4)
-            mma_16816(d, a, xr[2 * t], xr[2 * t + 1], d);
-        else
-            mma_16816(e, a, xr[2 * t], xr[2 * t + 1], e);
+#pragma unroll
+        for (int pp = 0; pp < MP; ++pp) {
+            if (t < 4)
+                mma_16816(d[pp], a, xr[pp][2 * t], xr[pp][2 * t + 1], d[pp]);
+            else
+                mma_16816(e[pp], a, xr[pp][2 * t], xr[pp][2 * t + 1], e[pp]);
+        }
     }
 }
 
@@ -217,9 +223,11 @@ __device__ __forceinline__ uint32_t load_scales(const M1& p, const uint16_t* sro
     return ldg_u16(q) | (ldg_u16(q + (2 * s + 1 < p.G ? 1 : 0)) << 16);
 }
 
+// MT: token slots (1, 2 or 4); tokens 2 pp and 2 pp + 1 share B operand pp.
 template <bool kEvenG, bool kWhole, bool kXEmb, int MT>
 __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
-    static_assert(MT == 1 || (MT == 2 && kWhole), "two tokens only with whole rows");
+    static_assert(MT == 1 || ((MT == 2 || MT == 4) && kWhole), "several tokens only with whole rows");
+    constexpr int MP = (MT + 1) / 2;  // B operands (token pairs)
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, tq = lane & 3;
@@ -418,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
             *reinterpret_cast<uint4*>(smem + tid * 256 + 16 * ((i + lane) & 7)) =
                 make_uint4(ent, ent, ent, ent);
     };
-    uint32_t xw[kUPW][16];  // whole rows: this warp's units never change, nor their x
+    uint32_t xw[kUPW][MP][16];  // whole rows: this warp's units never change, nor their x
     asm volatile("griddepcontrol.wait;" ::: "memory");
     {
         // Issue every global read of the set-up at once, then build the table
@@ -434,18 +442,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
 #pragma unroll
             for (int j = 0; j < kUPW; ++j) {
                 const int U = warp + kCW * j;
-                const bool act = U < upk && (g & 1) == (tq >> 1);
-                // two tokens: B columns 4-7 (lanes g >= 4) hold token 1
-                const uint16_t* xs = p.x + (MT == 2 ? (g >> 2) * p.K : 0) +
-                                     kSpan * (2 * U + ((g >> 1) & 1)) + 32 * tq;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                    if (act) v = ldg_v4_ordered(xs + 8 * q);
-                    xw[j][4 * q] = v.x;
-                    xw[j][4 * q + 1] = v.y;
-                    xw[j][4 * q + 2] = v.z;
-                    xw[j][4 * q + 3] = v.w;
+                for (int pp = 0; pp < MP; ++pp) {
+                    // B columns 0-3 (lanes g < 4) hold token 2 pp, columns 4-7
+                    // token 2 pp + 1
+                    const int tok = 2 * pp + (g >> 2);
+                    const bool act = U < upk && (g & 1) == (tq >> 1) && tok < p.M;
+                    const uint16_t* xs = p.x + static_cast<int64_t>(tok) * p.K +
+                                         kSpan * (2 * U + ((g >> 1) & 1)) + 32 * tq;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                        if (act) v = ldg_v4_ordered(xs + 8 * q);
+                        xw[j][pp][4 * q] = v.x;
+                        xw[j][pp][4 * q + 1] = v.y;
+                        xw[j][pp][4 * q + 2] = v.z;
+                        xw[j][pp][4 * q + 3] = v.w;
+                    }
                 }
             }
         } else {
@@ -462,7 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
 #pragma unroll
             for (int j = 0; j < kUPW; ++j)
 #pragma unroll
-                for (int i = 0; i < 16; ++i) xw[j][i] = cvt_bf16x2_f16x2(xw[j][i]);
+                for (int pp = 0; pp < MP; ++pp)
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) xw[j][pp][i] = cvt_bf16x2_f16x2(xw[j][pp][i]);
         } else {
             // x as binary16: 16-byte chunk (span s, quarter q, parity par, j)
             // holds x[128 s + 32 j + 8 q, +8) when par == j / 2 (the column
@@ -500,24 +515,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
 #pragma unroll
     for (int i = 0; i < kAhead; ++i) next_scales(sc[i]);
 
-    // One unit: two passes of eight MMAs; lane tq in {0, 1} adds span
-    // 2U + tq of rows g and g + 8, each group scaled by its own scale.
-    auto unit = [&](uint32_t a, const uint32_t (&xr)[16], const uint32_t (&s)[2], float& acc_lo,
-                    float& acc_hi) {
+    // One unit: two passes of eight MMAs per token pair; lane tq adds span
+    // 2U + (tq & 1) of rows g and g + 8 (token 2 pp + tq / 2), each group
+    // scaled by its own scale.
+    auto unit = [&](uint32_t a, const uint32_t (&xr)[MP][16], const uint32_t (&s)[2],
+                    float (&acc_lo)[MP], float (&acc_hi)[MP]) {
         const uint4 loA = lds128_ring<0>(a + offA), hiA = lds128_ring<0>(a + offA + rowhi);
         const uint4 loB = lds128_ring<0>(a + offB), hiB = lds128_ring<0>(a + offB + rowhi);
-        float dA[4] = {0.f, 0.f, 0.f, 0.f}, eA[4] = {0.f, 0.f, 0.f, 0.f};
-        float dB[4] = {0.f, 0.f, 0.f, 0.f}, eB[4] = {0.f, 0.f, 0.f, 0.f};
-        pass_mma(loA, hiA, xr, lane4_of(lane), dA, eA);
-        pass_mma(loB, hiB, xr, lane4_of(lane), dB, eB);
-        const float d0 = use_a ? dA[0] + eA[0] : dB[0] + eB[0];
-        const float d1 = use_a ? dA[1] + eA[1] : dB[1] + eB[1];
-        const float d2 = use_a ? dA[2] + eA[2] : dB[2] + eB[2];
-        const float d3 = use_a ? dA[3] + eA[3] : dB[3] + eB[3];
-        acc_lo = fmaf(f16_lo(s[0]), d0, acc_lo);
-        acc_lo = fmaf(f16_hi(s[0]), d1, acc_lo);
-        acc_hi = fmaf(f16_lo(s[1]), d2, acc_hi);
-        acc_hi = fmaf(f16_hi(s[1]), d3, acc_hi);
+        float dA[MP][4], eA[MP][4], dB[MP][4], eB[MP][4];
+#pragma unroll
+        for (int pp = 0; pp < MP; ++pp)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dA[pp][i] = eA[pp][i] = dB[pp][i] = eB[pp][i] = 0.f;
+        pass_mma<MP>(loA, hiA, xr, lane4_of(lane), dA, eA);
+        pass_mma<MP>(loB, hiB, xr, lane4_of(lane), dB, eB);
+        const float s0 = f16_lo(s[0]), s1 = f16_hi(s[0]), s2 = f16_lo(s[1]), s3 = f16_hi(s[1]);
+#pragma unroll
+        for (int pp = 0; pp < MP; ++pp) {
+            const float d0 = use_a ? dA[pp][0] + eA[pp][0] : dB[pp][0] + eB[pp][0];
+            const float d1 = use_a ? dA[pp][1] + eA[pp][1] : dB[pp][1] + eB[pp][1];
+            const float d2 = use_a ? dA[pp][2] + eA[pp][2] : dB[pp][2] + eB[pp][2];
+            const float d3 = use_a ? dA[pp][3] + eA[pp][3] : dB[pp][3] + eB[pp][3];
+            acc_lo[pp] = fmaf(s0, d0, acc_lo[pp]);
+            acc_lo[pp] = fmaf(s1, d1, acc_lo[pp]);
+            acc_hi[pp] = fmaf(s2, d2, acc_hi[pp]);
+            acc_hi[pp] = fmaf(s3, d3, acc_hi[pp]);
+        }
     };
     auto load_x = [&](uint32_t xa, uint32_t (&xr)[16]) {
         uint4 x0, x1, x2, x3;
@@ -553,7 +576,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
             started = true;
         }
         for (int t = pt0; t < pt1; ++t) {
-            float acc_lo = 0.f, acc_hi = 0.f;
+            float acc_lo[MP], acc_hi[MP];
+#pragma unroll
+            for (int pp = 0; pp < MP; ++pp) acc_lo[pp] = acc_hi[pp] = 0.f;
             for (int c = 0; c < (kWhole ? 1 : p.C); ++c) {
                 if (!bad && !mbar_wait(bars + 8u * slot, fparity)) {
                     bad = true;
@@ -567,9 +592,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
                         if (kWhole) {
                             unit(a0 + 128 * kCW * j, xw[j], sc[0][j], acc_lo, acc_hi);
                         } else {
-                            uint32_t xr[16];
+                            uint32_t xr[MP][16];
                             load_x(xlane + static_cast<uint32_t>(c * upk + warp + kCW * j) * (2 * kXSpan),
-                                   xr);
+                                   xr[0]);
                             unit(a0 + 128 * kCW * j, xr, sc[0][j], acc_lo, acc_hi);
                         }
                     }
@@ -590,15 +615,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
                 next_scales(sc[kAhead - 1]);
             }
             // lanes tq = 0, 1 hold the two spans' sums of rows g, g + 8 for
-            // token 0; lanes tq = 2, 3 the same for token 1 (columns 4-7)
-            acc_lo += __shfl_xor_sync(0xFFFFFFFFu, acc_lo, 1);
-            acc_hi += __shfl_xor_sync(0xFFFFFFFFu, acc_hi, 1);
-            if (tq == 0 || (MT == 2 && tq == 2)) {
-                // this warp's partials of the tile's rows:
-                // slot [tile][warp][token][row]
-                float* slot_w = acc_s + (((t - pt0) * kCW + warp) * MT + (tq >> 1)) * 16;
-                slot_w[g] = acc_lo;
-                slot_w[g + 8] = acc_hi;
+            // token 2 pp; lanes tq = 2, 3 the same for token 2 pp + 1
+#pragma unroll
+            for (int pp = 0; pp < MP; ++pp) {
+                acc_lo[pp] += __shfl_xor_sync(0xFFFFFFFFu, acc_lo[pp], 1);
+                acc_hi[pp] += __shfl_xor_sync(0xFFFFFFFFu, acc_hi[pp], 1);
+                const int tok = 2 * pp + (tq >> 1);
+                if ((tq & 1) == 0 && tok < MT) {
+                    // this warp's partials of the tile's rows:
+                    // slot [tile][warp][token][row]
+                    float* slot_w = acc_s + (((t - pt0) * kCW + warp) * MT + tok) * 16;
+                    slot_w[g] = acc_lo[pp];
+                    slot_w[g + 8] = acc_hi[pp];
+                }
             }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
@@ -607,6 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
             const int rl = r - 16 * pt0;
 #pragma unroll
             for (int tok = 0; tok < MT; ++tok) {
+                if (tok >= p.M) break;
                 const float* q = acc_s + ((rl >> 4) * kCW * MT + tok) * 16 + (rl & 15);
                 float sum = 0.f;
 #pragma unroll
@@ -649,8 +679,9 @@ cudaError_t take_gemv_m1_error(unsigned int* out) {
 cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int M, int64_t N, int64_t K, cudaStream_t s,
                            const DeviceInfo& dev) {
-    if (dev.smem_reserved != kBase || M < 1 || M > 2) return cudaErrorNotSupported;
+    if (dev.smem_reserved != kBase || M < 1 || M > 4) return cudaErrorNotSupported;
     M1 p{};
+    p.M = M;
     p.codes = codes;
     p.scales = scales;
     p.cb = cb;
@@ -666,7 +697,8 @@ cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const u
     // multiple of 128 bytes travel whole (a tile is one contiguous copy);
     // longer rows in C segments of KC bytes (a multiple of 128).
     const bool whole = p.rowbytes <= kMaxKC && p.rowbytes % 128 == 0;
-    if (M == 2 && !whole) return cudaErrorNotSupported;  // two tokens: whole rows only
+    if (M > 1 && !whole) return cudaErrorNotSupported;  // several tokens: whole rows only
+    const int mt = M == 1 ? 1 : (M == 2 ? 2 : 4);        // token slots
     if (whole) {
         p.C = 1;
         p.KC = p.rowbytes;
@@ -683,7 +715,7 @@ cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const u
     // up to kMaxPassTiles tiles (fewer passes, fewer barriers).
     auto layout = [&](int pt) {
         p.PT = pt;
-        p.bar_off = kAccOff + static_cast<uint32_t>(pt * M) * kTileSlotBytes;
+        p.bar_off = kAccOff + static_cast<uint32_t>(pt * mt) * kTileSlotBytes;
         p.x_off = p.bar_off + 128u;
         const uint32_t x_end = xemb ? p.x_off : p.x_off + static_cast<uint32_t>(p.SP) * 512u;
         p.ring_off = (x_end + 127u) & ~127u;
@@ -703,9 +735,12 @@ cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const u
     const int64_t tiles = (N + 15) / 16;
     const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
     const bool even = (p.G & 1) == 0;
-    if (whole && M == 2)
+    if (whole && mt == 2)
         return even ? launch_variant<true, true, true, 2>(p, grid, smem, 22, s, dev)
                     : launch_variant<false, true, true, 2>(p, grid, smem, 23, s, dev);
+    if (whole && mt == 4)
+        return even ? launch_variant<true, true, true, 4>(p, grid, smem, 24, s, dev)
+                    : launch_variant<false, true, true, 4>(p, grid, smem, 25, s, dev);
     if (whole) {
         return even ? launch_variant<true, true, true>(p, grid, smem, 16, s, dev)
                     : launch_variant<false, true, true>(p, grid, smem, 17, s, dev);

@@ -41,10 +41,10 @@ cudaError_t launch_dequant(const uint8_t* codes, const uint16_t* scales, const u
 cudaError_t launch_small_m(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int M, int64_t N, int64_t K,
                            cudaStream_t s, const DeviceInfo& dev);
-// M = 1 (and M = 2 with rows of at most 2 KB): bulk-copy-fed decode GEMV,
+// M = 1 (and M = 2..4 with rows of at most 2 KB): bulk-copy-fed decode GEMV,
 // one row range per CTA, launched with programmatic dependent launch.
 // Returns cudaErrorNotSupported when the shape does not fit it (K too large
-// for its shared-memory layout, or M = 2 with longer rows).
+// for its shared-memory layout, or M > 1 with longer rows).
 cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int M, int64_t N, int64_t K, cudaStream_t s,
                            const DeviceInfo& dev);
