@@ -208,6 +208,7 @@ def test_tiny_config_gemv():
     (2, 4096, 11008), (5, 257, 4160), (12, 1000, 2112), (7, 129, 320), (11, 2, 64),
     (13, 1, 64), (16, 129, 16448), (6, 4100, 2560), (10, 640, 7168),
     (20, 4096, 4160), (32, 200, 24576), (25, 1, 64),
+    (3, 17, 4096), (4, 1000, 2048), (2, 33, 256), (4, 1, 1024), (3, 2500, 3072),
     (17, 130, 512), (64, 257, 1088), (100, 96, 4096),
     (300, 200, 640), (257, 130, 2048), (48, 1000, 4160)])
 def test_ragged_shapes(M, N, K):
