@@ -1,4 +1,4 @@
-// q4_gemm_sm100.cu -- q4_gemm for M > 16 (prompt processing): a tcgen05
+// q4_gemm_sm100.cu -- q4_gemm for M > 32 (prompt processing): a tcgen05
 // tensor-core GEMM whose A operand is rebuilt from the 4-bit codes straight
 // into tensor memory.
 //
@@ -14,7 +14,8 @@
 // which keeps every output inside 1e-4 * sum|W x| + 1e-6 with a margin of
 // ~0.3 sqrt(K) standard deviations (about 20 at K = 4096).
 //
-// Roles (one CTA per tile of 128 weight rows x BMT tokens x one K chunk):
+// Roles (one CTA per tile of 128 weight rows -- two strips of 128 when
+// BMT <= 128 -- x BMT tokens x one K chunk):
 //  * warp 0 streams, by TMA, stages of 4 groups of codes (a 128-row x
 //    128-byte box, 128-byte swizzle) with their scales (cp.async);
 //  * warp 10 streams, by TMA, the x tile of every group (BMT tokens x 64 k
@@ -35,7 +36,11 @@
 // Measured on B200: with one thread issuing the MMAs, an x stream tied to the
 // weight stream and two commits per group, that thread spent most of each
 // group waiting for x and committing; the separate x warp and the shared
-// ring (one commit) keep the tensor pipe fed.
+// ring (one commit) keep the tensor pipe fed.  Each strip re-reads x from L2
+// (BMT x 128 bytes per group against 16 KB of codes per 4 groups), and an
+// SM takes in only about 50-65 GB/s: with two strips per tile every x tile
+// serves 256 rows (both accumulators fit in tensor memory up to BMT = 128),
+// which measured 1.2-1.3x faster at M = 40-128.
 // Every wait is bounded; a timeout sets an error bit, the roles drain what
 // they have in flight and the CTA frees its tensor memory before it exits.
 #include <mutex>
@@ -62,7 +67,13 @@ constexpr int kWStages = 2;
 // The A slots and the x stages form one ring: the MMA warp's one commit per
 // group frees both.
 constexpr uint32_t kTmemCols = 512;
-__device__ __forceinline__ uint32_t a_col(int slot) { return 256u + 32u * slot; }
+// Tensor-memory columns: accumulators in [0, 256) (strip h of a two-strip
+// tile at column 128 h), A slots in [256, 512): slot s of strip h at
+// 256 + 32 (kStrips s + h).
+template <int kStrips>
+__device__ __forceinline__ uint32_t a_col(int slot, int h) {
+    return 256u + 32u * static_cast<uint32_t>(kStrips * slot + h);
+}
 
 struct TcGemm {
     const uint16_t* scales;
@@ -101,10 +112,14 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
     return *reinterpret_cast<const uint32_t*>(&r);
 }
 
-template <bool kAsyncScales>
+// kStrips: 128-row strips per tile (2 only with BMT <= 128): both strips
+// share every x tile, which halves the x read per weight.
+template <bool kAsyncScales, int kStrips>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap xmap,
                    const TcGemm p) {
+    constexpr int kStageCode = kStrips * kWCodeBytes;
+    constexpr int kStageScale = kStrips * kWScaleBytes;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t base = smem_u32(smem);
@@ -121,10 +136,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + p.cb_off + 32);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + p.cb_off + 36);
 
-    // tile coordinates: blockIdx.x = ((strip * token_tiles) + tt) * ksplit + kc
+    // tile coordinates: blockIdx.x = ((tile * token_tiles) + tt) * ksplit + kc;
+    // the tile's first strip is kStrips * tile
     const int kc = blockIdx.x % p.ksplit;
     const int tt = (blockIdx.x / p.ksplit) % p.token_tiles;
-    const int strip = blockIdx.x / (p.ksplit * p.token_tiles);
+    const int strip = kStrips * (blockIdx.x / (p.ksplit * p.token_tiles));
     const int g_begin = kc * p.chunk_groups;
     const int g_end = min(p.G, g_begin + p.chunk_groups);
     const int ng = g_end - g_begin;  // groups of this CTA, >= 1
@@ -172,14 +188,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             const int g0 = g_begin + kWG * w;
-            const uint32_t cdst = base + kLutBytes + ws * kWCodeBytes;
-            const uint32_t sdst = base + p.wscale_off + ws * kWScaleBytes;
+            const uint32_t cdst = base + kLutBytes + ws * kStageCode;
+            const uint32_t sdst = base + p.wscale_off + ws * kStageScale;
             if (lane == 0) {
-                mbar_arrive_expect_tx(wfull(ws), kWCodeBytes);
-                tma_load_2d(cdst, &cmap, g0 * 32, strip * kR, wfull(ws));
+                mbar_arrive_expect_tx(wfull(ws), kStageCode);
+#pragma unroll
+                for (int h = 0; h < kStrips; ++h)
+                    tma_load_2d(cdst + h * kWCodeBytes, &cmap, g0 * 32, (strip + h) * kR, wfull(ws));
             }
 #pragma unroll
-            for (int jr = 0; jr < kR / 32; ++jr) {
+            for (int jr = 0; jr < kStrips * kR / 32; ++jr) {
                 const int r = lane + 32 * jr;
                 const int row = strip * kR + r;
                 if (kAsyncScales) {
@@ -251,8 +269,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint64_t bd = smem_desc_sw128(base + p.x_off + as * p.xstage_bytes, 1024);
 #pragma unroll
-                for (int t = 0; t < 4; ++t)
-                    tc_mma_ts(tmem, tmem + a_col(as) + 8 * t, bd + 2 * t, p.idesc, (gi > 0 || t > 0) ? 1u : 0u);
+                for (int h = 0; h < kStrips; ++h)
+#pragma unroll
+                    for (int t = 0; t < 4; ++t)
+                        tc_mma_ts(tmem + 128u * h, tmem + a_col<kStrips>(as, h) + 8 * t, bd + 2 * t,
+                                  p.idesc, (gi > 0 || t > 0) ? 1u : 0u);
                 tc_commit(gdone(as));  // frees the A slot and the x stage
             }
             if (ok) tc_commit(dfull);
@@ -294,22 +315,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = false;
                 break;
             }
-            const uint32_t rb = kLutBytes + ws * kWCodeBytes + row * 128;
             const int r8 = row & 7;
-            const uint4 c0 = ld_smem<uint4>(smem, rb + (((2 * j) ^ r8) << 4));
-            const uint4 c1 = ld_smem<uint4>(smem, rb + (((2 * j + 1) ^ r8) << 4));
-            const uint32_t sb = ld_smem<uint16_t>(smem, p.wscale_off + ws * kWScaleBytes + row * 8 + 2 * j);
-            const uint32_t s2 = sb | (sb << 16);
-            const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-            uint32_t h[32];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                h[4 * i + 0] = hmul2_u32(lut_at<0>(smem, wd[i], lane4), s2);
-                h[4 * i + 1] = hmul2_u32(lut_at<1>(smem, wd[i], lane4), s2);
-                h[4 * i + 2] = hmul2_u32(lut_at<2>(smem, wd[i], lane4), s2);
-                h[4 * i + 3] = hmul2_u32(lut_at<3>(smem, wd[i], lane4), s2);
+            for (int hs = 0; hs < kStrips; ++hs) {
+                const uint32_t rb = kLutBytes + ws * kStageCode + hs * kWCodeBytes + row * 128;
+                const uint4 c0 = ld_smem<uint4>(smem, rb + (((2 * j) ^ r8) << 4));
+                const uint4 c1 = ld_smem<uint4>(smem, rb + (((2 * j + 1) ^ r8) << 4));
+                const uint32_t sb = ld_smem<uint16_t>(
+                    smem, p.wscale_off + ws * kStageScale + hs * kWScaleBytes + row * 8 + 2 * j);
+                const uint32_t s2 = sb | (sb << 16);
+                const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                uint32_t h[32];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    h[4 * i + 0] = hmul2_u32(lut_at<0>(smem, wd[i], lane4), s2);
+                    h[4 * i + 1] = hmul2_u32(lut_at<1>(smem, wd[i], lane4), s2);
+                    h[4 * i + 2] = hmul2_u32(lut_at<2>(smem, wd[i], lane4), s2);
+                    h[4 * i + 3] = hmul2_u32(lut_at<3>(smem, wd[i], lane4), s2);
+                }
+                tc_st_x32(tlane + a_col<kStrips>(as, hs), h);
             }
-            tc_st_x32(tlane + a_col(as), h);
             tc_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -328,26 +353,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         // epilogue: each warpgroup writes half of the accumulator columns
         if (warp_wait(dfull, 0u, lane)) {
             tc_fence_after();
-            const int n = strip * kR + row;
             const int half = p.BMT / 2;
-            for (int c0 = wg * half; c0 < (wg + 1) * half; c0 += 8) {
-                uint32_t v[8];
-                asm volatile(
-                    "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                    : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-                      "=r"(v[7])
-                    : "r"(tlane + c0)
-                    : "memory");
-                tc_wait_ld();
+            for (int hs = 0; hs < kStrips; ++hs) {
+                const int n = (strip + hs) * kR + row;
+                for (int c0 = wg * half; c0 < (wg + 1) * half; c0 += 8) {
+                    uint32_t v[8];
+                    asm volatile(
+                        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                          "=r"(v[6]), "=r"(v[7])
+                        : "r"(tlane + 128u * hs + c0)
+                        : "memory");
+                    tc_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int m = tt * p.BMT + c0 + e;
-                    if (n < p.N && m < p.M) {
-                        float* dst = p.y + static_cast<long long>(m) * p.N + n;
-                        if (p.ksplit > 1)
-                            red_add_f32(dst, __uint_as_float(v[e]));
-                        else
-                            *dst = __uint_as_float(v[e]);
+                    for (int e = 0; e < 8; ++e) {
+                        const int m = tt * p.BMT + c0 + e;
+                        if (n < p.N && m < p.M) {
+                            float* dst = p.y + static_cast<long long>(m) * p.N + n;
+                            if (p.ksplit > 1)
+                                red_add_f32(dst, __uint_as_float(v[e]));
+                            else
+                                *dst = __uint_as_float(v[e]);
+                        }
                     }
                 }
             }
@@ -403,7 +430,10 @@ cudaError_t launch_prefill_tc(const uint8_t* codes, const uint16_t* scales, cons
     p.token_tiles = static_cast<int>((M + 255) / 256);
     p.BMT = static_cast<int>(((M + p.token_tiles - 1) / p.token_tiles + 15) / 16 * 16);
     const int strips = static_cast<int>((N + kR - 1) / kR);
-    const int tiles = strips * p.token_tiles;
+    // two strips per tile share each x tile when both accumulators fit
+    // (2 x BMT <= 256 tensor-memory columns)
+    const int nstrips = p.BMT <= 128 ? 2 : 1;
+    const int tiles = (strips + nstrips - 1) / nstrips * p.token_tiles;
     // K split: fewest waves x longest chunk (plus a fixed cost of ~4 groups),
     // one CTA per SM; ties go to the smaller split
     int ksplit = 1, chunk = (p.G + kWG - 1) / kWG * kWG;
@@ -424,8 +454,8 @@ cudaError_t launch_prefill_tc(const uint8_t* codes, const uint16_t* scales, cons
     p.chunk_groups = chunk;
     p.xstage_bytes = p.BMT * 128;
     p.idesc = idesc_f16_f32(kR, p.BMT);
-    p.wscale_off = kLutBytes + kWStages * kWCodeBytes;
-    p.x_off = (p.wscale_off + kWStages * kWScaleBytes + 1023) & ~1023;
+    p.wscale_off = kLutBytes + kWStages * nstrips * kWCodeBytes;
+    p.x_off = (p.wscale_off + kWStages * nstrips * kWScaleBytes + 1023) & ~1023;
     const int SX = kASlots;  // one x stage per A slot
     p.xstages = SX;
     p.cb_off = p.x_off + SX * p.xstage_bytes;
@@ -456,15 +486,25 @@ cudaError_t launch_prefill_tc(const uint8_t* codes, const uint16_t* scales, cons
         if (e != cudaSuccess) return e;
     }
     const bool async_scales = (p.G % kWG) == 0;
-    const void* fn = async_scales ? reinterpret_cast<const void*>(gemm_tc_kernel<true>)
-                                  : reinterpret_cast<const void*>(gemm_tc_kernel<false>);
-    e = ensure_smem_attr(fn, smem, 30 + (async_scales ? 0 : 1), dev.device);
+    const void* fn = nstrips == 2
+                         ? (async_scales ? reinterpret_cast<const void*>(gemm_tc_kernel<true, 2>)
+                                         : reinterpret_cast<const void*>(gemm_tc_kernel<false, 2>))
+                         : (async_scales ? reinterpret_cast<const void*>(gemm_tc_kernel<true, 1>)
+                                         : reinterpret_cast<const void*>(gemm_tc_kernel<false, 1>));
+    e = ensure_smem_attr(fn, smem, 30 + (async_scales ? 0 : 1) + 2 * (nstrips - 1), dev.device);
     if (e != cudaSuccess) return e;
     const int grid = tiles * ksplit;
-    if (async_scales)
-        gemm_tc_kernel<true><<<grid, kThreads, smem, s>>>(cmap, xmap, p);
-    else
-        gemm_tc_kernel<false><<<grid, kThreads, smem, s>>>(cmap, xmap, p);
+    if (nstrips == 2) {
+        if (async_scales)
+            gemm_tc_kernel<true, 2><<<grid, kThreads, smem, s>>>(cmap, xmap, p);
+        else
+            gemm_tc_kernel<false, 2><<<grid, kThreads, smem, s>>>(cmap, xmap, p);
+    } else {
+        if (async_scales)
+            gemm_tc_kernel<true, 1><<<grid, kThreads, smem, s>>>(cmap, xmap, p);
+        else
+            gemm_tc_kernel<false, 1><<<grid, kThreads, smem, s>>>(cmap, xmap, p);
+    }
     return cudaGetLastError();
 }
 
