@@ -30,7 +30,7 @@
  * cudaMalloc, ...).  The library keeps no pointer after a call returns and
  * holds only a per-device cache of the device's properties.  The one
  * allocation it makes is the stream-ordered scratch of the tensor-core path
- * of q4_gemm (M > 32; M = 17..32 only when the M <= 32 kernel declines a
+ * of q4_gemm (M > 24; M = 17..24 only when the M <= 24 kernel declines a
  * shape: 2 * M * K bytes for the binary16 copy of x), taken from a memory pool the
  * library creates once per device and returned to that pool on the same
  * stream before the call returns; the pool keeps the memory it has mapped.
@@ -137,10 +137,10 @@ q4_status q4_gemv(const uint8_t* codes, const uint16_t* scales,
  * Source: "deep-fold", "Method" table (prompt processing: a tensor-core NF4
  * GEMM that rebuilds weights into fragments); "Trapetum" overview, "What it
  * does" (speculative decoding verifies a few drafted tokens at once).
- * M <= 32 (verify batches, short prefill chunks) rebuilds binary16 codebook
+ * M <= 24 (verify batches, short prefill chunks) rebuilds binary16 codebook
  * values once per weight for all M tokens (mma.sync, tokens as columns):
  * exact products with binary32 accumulation, each group's sum scaled in
- * binary32, as q4_gemv.  M > 32 (prefill chunks) runs a tcgen05
+ * binary32, as q4_gemv.  M > 24 (prefill chunks) runs a tcgen05
  * tensor-core kernel: each weight is rebuilt as binary16(codebook * scale),
  * x is rounded to binary16, and products accumulate in binary32 in tensor
  * memory.  Either way the result is within 1e-4 * sum_k |W x| + 1e-6 of the
@@ -162,7 +162,7 @@ q4_status q4_gemm(const uint8_t* codes, const uint16_t* scales,
  * q4_gemm_noalloc -- q4_gemm for callers that may not allocate device memory.
  * The paper has no counterpart; this entry point exists for deployment.
  *
- * q4_gemm's tensor-core path (M > 32) takes 2 * M * K bytes of scratch from
+ * q4_gemm's tensor-core path (M > 24) takes 2 * M * K bytes of scratch from
  * a memory pool (see Ownership).  Some callers cannot let a library do that: engines that
  * reserve all device memory at start-up for a fixed arena and a KV cache
  * leave no headroom for a pool that grows later, and hosts that account for
@@ -175,8 +175,8 @@ q4_status q4_gemm(const uint8_t* codes, const uint16_t* scales,
  * Limits and hazards:
  *   - M > 16 needs 2 * M * K <= Q4_NOALLOC_SCRATCH_BYTES (e.g. M = 512 at
  *     K = 8192); larger inputs return Q4_ERR_TOO_LARGE before anything runs
- *     (for M = 17..32 this keeps room for the tensor-core path, which runs
- *     when the M <= 32 kernel declines a shape).  M <= 16 uses no scratch
+ *     (for M = 17..24 this keeps room for the tensor-core path, which runs
+ *     when the M <= 24 kernel declines a shape).  M <= 16 uses no scratch
  *     and has no such limit.
  *   - The array is shared by every call on a device and is not cleared
  *     between calls (each call overwrites what it reads).  Calls whose work
@@ -184,7 +184,7 @@ q4_status q4_gemm(const uint8_t* codes, const uint16_t* scales,
  *     -- race on it and may return wrong results; serialize them.
  *   - The first call that runs the tensor-core path on a device looks up the
  *     array's device address (a CUDA runtime query, no allocation) with that
- *     device current; make a first call with M > 32 before any stream
+ *     device current; make a first call with M > 24 before any stream
  *     capture.
  * Validation order: Q4_ERR_SHAPE, Q4_ERR_NULL, Q4_ERR_ALIGN (as q4_gemm), then
  * Q4_ERR_TOO_LARGE, Q4_ERR_ARCH, Q4_ERR_CUDA.
@@ -212,8 +212,8 @@ int q4_abi_version(void);
  * current device, stores the bits set since the last call in *flags and
  * clears them: bits 0-11 the M = 1 GEMV (bit 8: its shared-memory layout did
  * not match the device; bits 9-11: producer, drain and consumer waits), bits
- * 12-15 the M = 2..32 kernel (the same four conditions), bits 16-31 the
- * M > 32 tensor-core GEMM; 0 = none.  Not an operation of the method; a
+ * 12-15 the M = 2..24 kernel (the same four conditions), bits 16-31 the
+ * tensor-core GEMM (M > 24); 0 = none.  Not an operation of the method; a
  * health check.
  * Returns Q4_ERR_NULL for a NULL flags, Q4_ERR_CUDA if a CUDA call fails.
  */

@@ -171,9 +171,9 @@ q4_status q4_gemm(const uint8_t* codes, const uint16_t* scales, const uint16_t* 
     if (M <= 16)
         return after_launch(
             launch_small_m(codes, scales, codebook, x, y, static_cast<int>(M), N, K, stream, dev));
-    if (M <= 32) {
+    if (M <= 24) {
         // still weight-streaming: the CUDA-core decode kernel beats the
-        // tensor-core pipeline here (its per-group MMA issue does not shrink with M)
+        // tensor-core pipeline up to 24 tokens (measured crossover on B200)
         cudaError_t e = launch_gemm_small(codes, scales, codebook, x, y, static_cast<int>(M), N, K,
                                           stream, dev);
         if (e != cudaErrorNotSupported) return after_launch(e);
@@ -196,7 +196,7 @@ q4_status q4_gemm_noalloc(const uint8_t* codes, const uint16_t* scales, const ui
     if (M <= 16)
         return after_launch(
             launch_small_m(codes, scales, codebook, x, y, static_cast<int>(M), N, K, stream, dev));
-    if (M <= 32) {
+    if (M <= 24) {
         cudaError_t e = launch_gemm_small(codes, scales, codebook, x, y, static_cast<int>(M), N, K,
                                           stream, dev);
         if (e != cudaErrorNotSupported) return after_launch(e);

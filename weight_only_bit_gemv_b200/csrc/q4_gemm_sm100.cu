@@ -1,4 +1,4 @@
-// q4_gemm_sm100.cu -- q4_gemm for M > 32 (prompt processing): a tcgen05
+// q4_gemm_sm100.cu -- q4_gemm for M > 24 (prompt processing): a tcgen05
 // tensor-core GEMM whose A operand is rebuilt from the 4-bit codes straight
 // into tensor memory.
 //

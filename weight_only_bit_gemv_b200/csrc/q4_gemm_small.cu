@@ -1,5 +1,6 @@
 // q4_gemm_small.cu -- q4_gemm for M = 2..32 tokens (verify batches, short
-// prefill chunks) on sm_100a.
+// prefill chunks) on sm_100a; q4_gemm sends it M <= 24 (above that the
+// two-strip tensor-core kernel streams faster).
 //
 // What it computes: y[m][n] = sum_g scale[n][g] * sum_{k in g} cb[code(n,k)] * x[m][k]
 // ("deep-fold", "Method": 64-weight groups, four-bit codes, one FP16 scale,
