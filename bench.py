@@ -359,6 +359,7 @@ def run_ours(args, world, rank, local):
     # ---- other workloads: a full 8B decode step, small-M verify batches --------
     step8b = None if args.no_step else bench_decode_step(dev, cb, stream, hbm_peak)
     smallm = None if args.no_smallm else bench_small_m(dev, cb, stream, hbm_peak)
+    embed = None if args.no_smallm else bench_embed_rows(dev, cb, stream, hbm_peak)
 
     # ---- CPU baseline: the oracle on the host --------------------------------
     cpu = None
@@ -423,6 +424,8 @@ def run_ours(args, world, rank, local):
         line["decode_step_llama31_8b"] = step8b
     if smallm is not None:
         line["small_m_verify"] = smallm
+    if embed is not None:
+        line["embed_rows"] = embed
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if rank == 0:
@@ -600,6 +603,50 @@ def bench_small_m(dev, cb, stream, hbm_peak, Ms=(2, 4, 8, 16), reps=20):
     torch.cuda.empty_cache()
     return {"workload": "small_m_verify: Llama-3.1-8B qkv, o, gate_up, down + lm_head, q4_gemm per "
                         "linear, 5 launches in one CUDA graph", **out}
+
+
+def bench_embed_rows(dev, cb, stream, hbm_peak, n_ids=4096, reps=20):
+    """q4_embed_rows on the Llama-3.1-8B embedding table (128256 x 4096,
+    packed: 279 MB, more than L2): a prefill chunk of ``n_ids`` seeded token
+    ids, four calls per CUDA graph."""
+    import torch
+    import weight_only_bit_gemv_b200 as q4
+    N, K = 128256, 4096
+    w = synth.weights_device(synth.seed_for(9, 0, "embed"), N, K, 0.02, dev)
+    codes, scales = q4.q4_pack(w, cb)
+    del w
+    g_ids = torch.Generator(device="cpu").manual_seed(12345)
+    ids = torch.randint(0, N, (4, n_ids), generator=g_ids, dtype=torch.int32).to(dev)
+    outs = [torch.empty((n_ids, K), dtype=torch.float32, device=dev) for _ in range(4)]
+    with torch.cuda.stream(stream):
+        for j in range(4):
+            q4.q4_embed_rows(codes, scales, cb, ids[j], outs[j])
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for j in range(4):
+            q4.q4_embed_rows(codes, scales, cb, ids[j], outs[j])
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / (reps * 4)
+    # algorithmic bytes: each id's code row and scales read, its fp32 row
+    # written, the id itself and the codebook
+    nbytes = n_ids * (K // 2 + (K // GROUP) * 2 + 4 * K + 4) + 32
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del g, codes, scales, outs
+    torch.cuda.empty_cache()
+    return {"workload": f"llama31_8b embedding table {N}x{K}, {n_ids} seeded token ids per call",
+            "us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
+            "hbm_frac_of_measured": round(gbs / hbm_peak, 4),
+            "timing": "CUDA graph of 4 calls on different ids, replayed 20 times"}
 
 
 def cpu_baseline(lins, cb, seconds):

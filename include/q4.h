@@ -110,6 +110,25 @@ q4_status q4_dequant(const uint8_t* codes, const uint16_t* scales,
                      int64_t K, q4_stream_t stream);
 
 /*
+ * q4_embed_rows -- dequantize only the requested rows of a packed matrix
+ * (an embedding table): out[i][k] = codebook[code(ids[i], k)] *
+ * scale[ids[i]][k / 64] in binary32, exact, as q4_dequant.
+ * Source: "deep-fold", introduction and Figure 1 (embeddings, PackedEmbed,
+ * decode only the requested rows, on a path of their own).
+ * ids[i] outside [0, N) writes a row of zeros (ids live in device memory, so
+ * they are not checked on the host).  Rows may repeat.
+ * In: codes [N][K/2], scales [N][K/64], codebook, ids [n_ids] int32.
+ * Out: out [n_ids][K] fp32.
+ * Validation: Q4_ERR_SHAPE for a bad K (as q4_dequant), N or n_ids outside
+ * [0, Q4_MAX_MN]; n_ids == 0 returns Q4_OK without a launch; then
+ * Q4_ERR_NULL, Q4_ERR_ALIGN (every pointer 16-byte aligned), Q4_ERR_ARCH,
+ * Q4_ERR_CUDA.
+ */
+q4_status q4_embed_rows(const uint8_t* codes, const uint16_t* scales,
+                        const uint16_t* codebook, const int32_t* ids, float* out,
+                        int64_t n_ids, int64_t N, int64_t K, q4_stream_t stream);
+
+/*
  * q4_gemv -- one-token decode: y[0][n] = sum_k W[n][k] * x[0][k], M must be 1.
  * Source: "deep-fold", "Method" table (decode: a CUDA-core NF4 GEMV that
  * rebuilds values while it multiplies); "Trapetum" overview, "The bandwidth

@@ -100,6 +100,8 @@ class Oracle:
         lib.oracle_dequant.argtypes = [P, P, P, P, I64, I64]
         lib.oracle_matmul.restype = ctypes.c_int
         lib.oracle_matmul.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P, P]
+        lib.oracle_embed_rows.restype = ctypes.c_int
+        lib.oracle_embed_rows.argtypes = [P, P, P, P, I64, I64, I64, P]
         self.lib = lib
         self.path = path
 
@@ -157,6 +159,19 @@ class Oracle:
             raise ValueError("oracle_dequant: bad shape")
         return out
 
+    def embed_rows(self, codes, scales, cb, ids) -> np.ndarray:
+        """Rows ``ids`` (int32) of the dequantized matrix, fp32 [n, K]; ids
+        outside [0, N) give rows of zeros."""
+        codes, scales, cb = _c(codes, np.uint8), _c(scales, np.uint16), _c(cb, np.uint16)
+        ids = _c(np.asarray(ids, dtype=np.int32), np.int32)
+        N, K = codes.shape[0], codes.shape[1] * 2
+        out = np.empty((ids.size, K), np.float32)
+        rc = self.lib.oracle_embed_rows(_ptr(codes), _ptr(scales), _ptr(cb), _ptr(ids), ids.size,
+                                        N, K, _ptr(out))
+        if rc != 0:
+            raise ValueError("oracle_embed_rows: bad shape")
+        return out
+
     def matmul(self, codes, scales, cb, x, rows=None, with_abs: bool = True):
         """y [M, n_out] (fp32) and sum|W*x| [M, n_out] (fp64, or None).
 
@@ -201,3 +216,4 @@ def weight(codes, scales, cb, n, k): return default().weight(codes, scales, cb, 
 def dequant(codes, scales, cb): return default().dequant(codes, scales, cb)
 def matmul(codes, scales, cb, x, rows=None, with_abs=True):
     return default().matmul(codes, scales, cb, x, rows, with_abs)
+def embed_rows(codes, scales, cb, ids): return default().embed_rows(codes, scales, cb, ids)

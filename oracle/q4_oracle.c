@@ -17,6 +17,8 @@
  *    payload is about 3.76x smaller than BF16; kernels rebuild the values as
  *    they multiply.  Same page, "Method" table: decode is a GEMV, prefill a
  *    tensor-core GEMM.
+ *  - Same page, introduction and Figure 1: embeddings (PackedEmbed) decode
+ *    only the requested rows, on a path of their own.
  *  - "Trapetum" overview, "What it does": the fused kernel reads the weights
  *    straight out of the codebook.  "Trapetum" landing page: the matrix is
  *    decoded inside the matmul and never materialized.
@@ -35,7 +37,9 @@
  *  - dequantized weight W = cb[code] * scale in binary32 (exact: an 11-bit by
  *    11-bit significand product);
  *  - matmul reference: the products W * x summed in fp64 in increasing k and
- *    rounded once to binary32.
+ *    rounded once to binary32;
+ *  - embedding rows: the requested rows of the dequantized matrix in binary32;
+ *    an id outside [0, N) gives a row of zeros.
  */
 #include "q4_oracle.h"
 
@@ -261,6 +265,23 @@ int oracle_dequant(const uint8_t* codes, const uint16_t* scales,
     for (int64_t n = 0; n < N; ++n)
         for (int64_t k = 0; k < K; ++k)
             w_out[n * K + k] = oracle_weight(codes, scales, cb, K, n, k);
+    return 0;
+}
+
+/* Embedding rows ("deep-fold", introduction and Figure 1: embeddings decode
+ * only the requested rows): out[i] = row ids[i] of the dequantized matrix,
+ * a row of zeros for an id outside [0, N). */
+int oracle_embed_rows(const uint8_t* codes, const uint16_t* scales,
+                      const uint16_t* cb, const int32_t* ids, int64_t n_ids,
+                      int64_t N, int64_t K, float* out)
+{
+    if (n_ids < 0 || N < 0 || K <= 0 || K % ORACLE_GROUP != 0)
+        return -1;
+    for (int64_t i = 0; i < n_ids; ++i) {
+        int64_t n = ids[i];
+        for (int64_t k = 0; k < K; ++k)
+            out[i * K + k] = (n >= 0 && n < N) ? oracle_weight(codes, scales, cb, K, n, k) : 0.0f;
+    }
     return 0;
 }
 

@@ -50,6 +50,12 @@ float    oracle_weight(const uint8_t* codes, const uint16_t* scales,
 int      oracle_dequant(const uint8_t* codes, const uint16_t* scales,
                         const uint16_t* cb, float* w_out, int64_t N, int64_t K);
 
+/* rows ids[i] of the dequantized matrix into out [n_ids][K]; ids outside
+ * [0, N) give rows of zeros.  Returns 0 or -1. */
+int      oracle_embed_rows(const uint8_t* codes, const uint16_t* scales,
+                           const uint16_t* cb, const int32_t* ids, int64_t n_ids,
+                           int64_t N, int64_t K, float* out);
+
 /* y[m][i] = sum_k W[n_i][k] * x[m][k] in fp64, rounded once to fp32, and
  * absacc[m][i] = sum_k |W[n_i][k] * x[m][k]| in fp64.
  * rows == NULL: n_i = i for i < N and the outputs are [M][N];

@@ -94,6 +94,18 @@ def test_pack_dequant_reject(lib):
     assert lib.q4_dequant(A, A, A, A, 0, 64, None) == OK
 
 
+def test_embed_rows_rejects(lib):
+    f = lib.q4_embed_rows
+    assert f(A, A, A, A, A, 4, 64, 100, None) == SHAPE        # K % 64
+    assert f(A, A, A, A, A, -1, 64, 64, None) == SHAPE        # n_ids < 0
+    assert f(A, A, A, A, A, 4, -1, 64, None) == SHAPE         # N < 0
+    assert f(None, None, None, None, None, 0, 64, 64, None) == OK   # no ids: no launch
+    assert f(A, A, A, None, A, 4, 64, 64, None) == NULL       # ids
+    assert f(A, A, A, A, None, 4, 64, 64, None) == NULL       # out
+    assert f(A, A, A, MIS, A, 4, 64, 64, None) == ALIGN
+    assert f(A, A, A, A, MIS, 4, 64, 64, None) == ALIGN
+
+
 def test_binding_marshalling_checks():
     import torch
     cpu = torch.zeros(4, 32, dtype=torch.uint8)

@@ -88,6 +88,25 @@ def gpu_dequant(codes, scales, cb):
     return w.cpu().numpy()
 
 
+@pytest.mark.parametrize("N,K,n_ids", [(32000, 4096, 64), (37, 192, 9), (1, 64, 3), (513, 1088, 0)])
+def test_embed_rows_bit_exact(N, K, n_ids):
+    """Embedding rows: bit-exact against the oracle, with repeated ids, both
+    ends of the table and ids outside [0, N) (rows of zeros)."""
+    codes, scales = random_packed(31 + N, N, K)
+    rng = np.random.default_rng(N + K)
+    ids = rng.integers(0, N, size=n_ids).astype(np.int32)
+    if n_ids >= 3:
+        ids[:3] = [0, N - 1, -5]
+    if n_ids >= 6:
+        ids[3:6] = [N, ids[0], 1 << 30]
+    out = q4.q4_embed_rows(dev_u8(codes), dev_u16(scales), dev_u16(NF4),
+                           torch.from_numpy(ids).cuda())
+    torch.cuda.synchronize()
+    ref = oracle.embed_rows(codes, scales, NF4, ids)
+    assert out.shape == (n_ids, K)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
 @pytest.mark.parametrize("N,K", [(128, 256), (1, 64), (37, 448), (300, 4096)])
 def test_pack_dequant_bit_exact(N, K):
     w = synth.weights(7 + N, N, K, 0.02)

@@ -366,6 +366,29 @@ def pin_matmul_row_subset(o):
     assert np.array_equal(ys, y[:, rows]) and np.array_equal(as_, a[:, rows])
 
 
+def pin_embed_rows_definition(o):
+    """Embedding rows ("deep-fold", introduction and Figure 1: only the
+    requested rows are decoded): each output row equals cb[code] * scale of
+    that row, computed here from the bytes with numpy's own binary16 ->
+    binary32 conversion and binary32 product; ids outside [0, N) give zeros;
+    repeated ids repeat the row."""
+    rng = np.random.default_rng(12)
+    N, K = 23, 3 * GROUP
+    codes = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    scales = synth.f32_to_f16_bits(rng.uniform(0.005, 0.05, size=(N, K // GROUP)).astype(np.float32))
+    ids = np.array([5, 0, 22, -1, 23, 5, 1 << 30, 11], np.int32)
+    got = o.embed_rows(codes, scales, NF4, ids)
+    cbf = NF4.view(np.float16).astype(np.float32)
+    sf = scales.view(np.float16).astype(np.float32)
+    lo, hi = codes & 0x0F, codes >> 4
+    nib = np.empty((N, K), np.uint8)
+    nib[:, 0::2], nib[:, 1::2] = lo, hi
+    w = cbf[nib] * np.repeat(sf, GROUP, axis=1)
+    for i, n in enumerate(ids):
+        want = w[n] if 0 <= n < N else np.zeros(K, np.float32)
+        assert np.array_equal(got[i], want), f"row {i} (id {n})"
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
@@ -429,6 +452,10 @@ MUTANTS = {
     "nf4_neg_spacing": ("(double)i / 7.0", "(double)i / 8.0"),
     "divide_becomes_multiply": ("float r = wg[j] / s;", "float r = wg[j] * s;"),
     "abs_sum_signed": ("aacc += fabs(p);", "aacc += p;"),
+    "embed_out_of_range_clamped": ("(n >= 0 && n < N) ? oracle_weight(codes, scales, cb, K, n, k) : 0.0f",
+                                   "oracle_weight(codes, scales, cb, K, n < 0 ? 0 : (n >= N ? N - 1 : n), k)"),
+    "embed_row_off_by_one": ("? oracle_weight(codes, scales, cb, K, n, k)",
+                             "? oracle_weight(codes, scales, cb, K, n > 0 ? n - 1 : 0, k)"),
 }
 
 

@@ -61,7 +61,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.q4_gemv.argtypes = [P, P, P, P, P, I64, I64, I64, S]
     lib.q4_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, S]
     lib.q4_gemm_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, S]
-    for f in ("q4_pack", "q4_dequant", "q4_gemv", "q4_gemm", "q4_gemm_noalloc"):
+    lib.q4_embed_rows.argtypes = [P, P, P, P, P, I64, I64, I64, S]
+    for f in ("q4_pack", "q4_dequant", "q4_gemv", "q4_gemm", "q4_gemm_noalloc", "q4_embed_rows"):
         getattr(lib, f).restype = ctypes.c_int
     lib.q4_status_string.argtypes = [ctypes.c_int]
     lib.q4_status_string.restype = ctypes.c_char_p
@@ -159,6 +160,27 @@ def q4_dequant(codes: torch.Tensor, scales: torch.Tensor, codebook: torch.Tensor
     return w_out
 
 
+def q4_embed_rows(codes: torch.Tensor, scales: torch.Tensor, codebook: torch.Tensor,
+                  ids: torch.Tensor, out: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """out [n, K] fp32 = rows ids [n] (int32) of the packed matrix, dequantized
+    exactly; ids outside [0, N) give rows of zeros."""
+    N, K = _packed_dims(codes)
+    if ids.dim() != 1:
+        raise ValueError("ids must be [n]")
+    n = ids.shape[0]
+    if out is None:
+        out = torch.empty((n, K), dtype=torch.float32, device=codes.device)
+    _need(codes, "codes", (torch.uint8,))
+    _need(scales, "scales", _H16, (N, K // GROUP))
+    _need(codebook, "codebook", _H16, (16,))
+    _need(ids, "ids", (torch.int32,))
+    _need(out, "out", (torch.float32,), (n, K))
+    st = load().q4_embed_rows(codes.data_ptr(), scales.data_ptr(), codebook.data_ptr(),
+                              ids.data_ptr(), out.data_ptr(), n, N, K, _stream(codes, stream))
+    _check(st, "q4_embed_rows")
+    return out
+
+
 def _matmul(fn: str, codes, scales, codebook, x, y, stream):
     N, K = _packed_dims(codes)
     if x.dim() != 2 or x.shape[1] != K:
@@ -183,7 +205,8 @@ def q4_gemv(codes, scales, codebook, x, y=None, stream=None) -> torch.Tensor:
 
 
 def q4_gemm(codes, scales, codebook, x, y=None, stream=None) -> torch.Tensor:
-    """y [M, N] = x [M, K] @ W^T for any M (M <= 16: verify batches; M > 16: prefill)."""
+    """y [M, N] = x [M, K] @ W^T for any M (M <= 24: verify batches and short
+    chunks on the CUDA-core decode kernels; M > 24: prefill on tensor cores)."""
     return _matmul("q4_gemm", codes, scales, codebook, x, y, stream)
 
 

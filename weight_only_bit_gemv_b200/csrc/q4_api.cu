@@ -148,6 +148,22 @@ q4_status q4_dequant(const uint8_t* codes, const uint16_t* scales, const uint16_
     return after_launch(launch_dequant(codes, scales, codebook, w_out, N, K, stream, dev));
 }
 
+q4_status q4_embed_rows(const uint8_t* codes, const uint16_t* scales, const uint16_t* codebook,
+                        const int32_t* ids, float* out, int64_t n_ids, int64_t N, int64_t K,
+                        q4_stream_t stream) {
+    q4_status st = check_K(K);
+    if (st != Q4_OK) return st;
+    if (N < 0 || N > Q4_MAX_MN || n_ids < 0 || n_ids > Q4_MAX_MN) return Q4_ERR_SHAPE;
+    if (n_ids == 0) return Q4_OK;
+    if (!codes || !scales || !codebook || !ids || !out) return Q4_ERR_NULL;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(codebook) || !aligned16(ids) ||
+        !aligned16(out))
+        return Q4_ERR_ALIGN;
+    DeviceInfo dev;
+    if ((st = gate(&dev)) != Q4_OK) return st;
+    return after_launch(launch_embed_rows(codes, scales, codebook, ids, out, n_ids, N, K, stream, dev));
+}
+
 q4_status q4_gemv(const uint8_t* codes, const uint16_t* scales, const uint16_t* codebook,
                   const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
                   q4_stream_t stream) {

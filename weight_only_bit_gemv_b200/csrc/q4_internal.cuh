@@ -37,6 +37,9 @@ cudaError_t launch_pack(const float* w, const uint16_t* cb, uint8_t* codes, uint
                         int64_t N, int64_t K, cudaStream_t s, const DeviceInfo& dev);
 cudaError_t launch_dequant(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            float* w, int64_t N, int64_t K, cudaStream_t s, const DeviceInfo& dev);
+cudaError_t launch_embed_rows(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                             const int32_t* ids, float* out, int64_t n_ids, int64_t N, int64_t K,
+                             cudaStream_t s, const DeviceInfo& dev);
 // M in [1, 16]: decoded codebook values on mma.sync, exact products, fp32 sums.
 cudaError_t launch_small_m(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int M, int64_t N, int64_t K,

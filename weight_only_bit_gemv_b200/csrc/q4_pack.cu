@@ -10,6 +10,9 @@
 // bit-identical to any serial IEEE implementation of the same steps.
 //
 // Dequant writes W = codebook[code] * scale in binary32, which is exact.
+// Embed-rows writes the same values for the requested rows only ("deep-fold",
+// introduction and Figure 1: embeddings decode only the requested rows, on a
+// path of their own).
 #include "q4_internal.cuh"
 
 namespace q4 {
@@ -142,10 +145,60 @@ cudaError_t launch_pack(const float* w, const uint16_t* cb, uint8_t* codes, uint
     return cudaGetLastError();
 }
 
+// Row ids[i] of the packed matrix, dequantized into out[i]; ids outside
+// [0, N) give a row of zeros.  A thread writes 16 consecutive values (one
+// 8-byte code load, four 16-byte stores), so a warp's stores are contiguous.
+__global__ void __launch_bounds__(256) embed_rows_kernel(const uint8_t* __restrict__ codes,
+                                                         const uint16_t* __restrict__ scales,
+                                                         const uint16_t* __restrict__ cb,
+                                                         const int32_t* __restrict__ ids,
+                                                         float* __restrict__ out, int64_t n_ids,
+                                                         int64_t N, int64_t K) {
+    __shared__ float cbf[16];
+    if (threadIdx.x < 16) cbf[threadIdx.x] = half_bits_to_float(cb[threadIdx.x]);
+    __syncthreads();
+    const int64_t per_row = K / 16;
+    const int64_t total = n_ids * per_row;
+    const int64_t G = K / kGroup;
+    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+         idx += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = idx / per_row, j = idx - i * per_row;
+        const int64_t k0 = j * 16;
+        const int64_t n = __ldg(ids + i);
+        float v[16];
+        if (n >= 0 && n < N) {
+            const uint2 b = __ldg(reinterpret_cast<const uint2*>(codes + n * (K / 2) + j * 8));
+            const float sc = half_bits_to_float(scales[n * G + k0 / kGroup]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t word = (e < 4) ? b.x : b.y;
+                const uint32_t code = (word >> (8 * (e % 4))) & 0xFFu;
+                v[2 * e] = __fmul_rn(cbf[code & 0xF], sc);
+                v[2 * e + 1] = __fmul_rn(cbf[code >> 4], sc);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = 0.f;
+        }
+        float4* dst = reinterpret_cast<float4*>(out + i * K + k0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+}
+
 cudaError_t launch_dequant(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            float* w, int64_t N, int64_t K, cudaStream_t s, const DeviceInfo& dev) {
     const int64_t items = N * (K / 16);
     dequant_kernel<<<grid_for(items, 256, dev), 256, 0, s>>>(codes, scales, cb, w, N, K);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_embed_rows(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                             const int32_t* ids, float* out, int64_t n_ids, int64_t N, int64_t K,
+                             cudaStream_t s, const DeviceInfo& dev) {
+    const int64_t items = n_ids * (K / 16);
+    embed_rows_kernel<<<grid_for(items, 256, dev), 256, 0, s>>>(codes, scales, cb, ids, out, n_ids, N,
+                                                               K);
     return cudaGetLastError();
 }
 
