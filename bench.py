@@ -58,8 +58,8 @@ def peaks():
 # (4096 -> 22016) from an ncu capture, with the SHA-1 of the kernel source it
 # was taken on; when the source changes the figure no longer applies and the
 # bench reports null.
-GEMV_TRAFFIC = {"bytes": 47955456 + 7424,
-                "source_sha1": "2eb9fe7336999dcb01cf1a56090cc2589e16c70a",
+GEMV_TRAFFIC = {"bytes": 47952128 + 7680,
+                "source_sha1": "1da9f429fe162a2b3c7c184dc784cef12b76512d",
                 "capture": "ncu --set full --clock-control none -k regex:gemv_m1 -s 2 -c 1 "
                            "python -m weight_only_bit_gemv_b200.profile_case --M 1 --iters 5 "
                            "--copies 2 --workload llama2_7b_layer --linear gate_up"}
