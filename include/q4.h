@@ -213,6 +213,47 @@ q4_status q4_gemm_noalloc(const uint8_t* codes, const uint16_t* scales,
                           const uint16_t* codebook, const uint16_t* x, float* y,
                           int64_t M, int64_t N, int64_t K, q4_stream_t stream);
 
+/*
+ * CopyRing -- matmuls whose packed weights live in host memory.
+ * Source: "deep-fold", "Method" table (models that exceed the GPU budget:
+ * selected packed matrices stream from pinned host memory through two
+ * reusable GPU slots) and Figure 1 (overflow adds pinned host storage and two
+ * reusable device slots, then the same GEMM kernel).
+ *
+ * q4_ring_create -- on the current device, allocate two device slots of
+ * slot_bytes each (cudaMalloc), a copy stream and four events.  A slot must
+ * hold a matrix's codes, padded to 256 bytes, plus its scales:
+ * ceil(N * K / 2 / 256) * 256 + N * K / 32 bytes.  Returns Q4_ERR_NULL for a
+ * NULL ring, Q4_ERR_SHAPE for slot_bytes <= 0, Q4_ERR_ARCH, Q4_ERR_CUDA.
+ *
+ * q4_ring_gemm -- y = x W^T exactly as q4_gemm (q4_gemv's kernel for M = 1),
+ * with codes [N][K/2] and scales [N][K/64] in host memory.  The call
+ * enqueues, without blocking the host:
+ *   1. on the ring's copy stream, once the matmul that last read the ring's
+ *      next slot has finished, the copy of codes and scales into that slot;
+ *   2. on `stream`, once that copy has landed, the matmul on the slot.
+ * Consecutive calls alternate the slots, so the copy of one call overlaps the
+ * matmul of the one before.  Use page-locked host memory (cudaHostAlloc or
+ * cudaHostRegister); pageable memory is correct but does not overlap.  The
+ * host buffers must stay unchanged until the call's copy has run
+ * (synchronize `stream`).  Calls on one ring are serialized by a mutex; each
+ * must be made with the ring's device current (else Q4_ERR_CUDA,
+ * cudaErrorInvalidDevice).  Validation as q4_gemm (the host pointers must be
+ * 16-byte aligned), plus Q4_ERR_NULL for a NULL ring and Q4_ERR_TOO_LARGE
+ * for a matrix larger than a slot.  Not capturable in a CUDA graph (it
+ * records events on a stream of its own).
+ *
+ * q4_ring_destroy -- wait for the ring's copies and the matmuls that read its
+ * slots, then free it.
+ */
+typedef struct q4_ring q4_ring;
+q4_status q4_ring_create(int64_t slot_bytes, q4_ring** ring);
+q4_status q4_ring_gemm(q4_ring* ring, const uint8_t* host_codes,
+                       const uint16_t* host_scales, const uint16_t* codebook,
+                       const uint16_t* x, float* y, int64_t M, int64_t N,
+                       int64_t K, q4_stream_t stream);
+q4_status q4_ring_destroy(q4_ring* ring);
+
 /* Human-readable name of a status code (static storage, never NULL). */
 const char* q4_status_string(q4_status status);
 

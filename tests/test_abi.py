@@ -106,6 +106,15 @@ def test_embed_rows_rejects(lib):
     assert f(A, A, A, A, MIS, 4, 64, 64, None) == ALIGN
 
 
+def test_ring_rejects(lib):
+    import ctypes
+    h = ctypes.c_void_p()
+    assert lib.q4_ring_create(1 << 20, None) == NULL
+    assert lib.q4_ring_create(0, ctypes.byref(h)) == SHAPE
+    assert lib.q4_ring_gemm(None, A, A, A, A, A, 1, 64, 64, None) == NULL
+    assert lib.q4_ring_destroy(None) == NULL
+
+
 def test_binding_marshalling_checks():
     import torch
     cpu = torch.zeros(4, 32, dtype=torch.uint8)

@@ -313,6 +313,38 @@ def test_llama2_70b_prefill(linear, M):
     assert_close(y, codes, scales, NF4, x, rows=rows, label=f"{linear} M={M}")
 
 
+def test_ring_streams_host_weights():
+    """CopyRing: packed weights in pinned host memory give the y of the
+    resident path (bit for bit at M = 1) and stay within the tolerance of the
+    oracle, over a sequence that reuses both slots."""
+    shapes = [(300, 4096), (1000, 2048), (37, 448), (512, 4096), (129, 1088)]
+    packs = [random_packed(90 + i, N, K) for i, (N, K) in enumerate(shapes)]
+    ring = q4.Ring(max(q4.ring_slot_bytes(N, K) for N, K in shapes))
+    try:
+        for M in (1, 4):
+            outs = []
+            for (N, K), (codes, scales) in zip(shapes, packs):
+                ch = torch.from_numpy(codes).pin_memory()
+                sh = torch.from_numpy(scales.view(np.int16)).pin_memory()
+                x = synth.activations(N + K + M, M, K)
+                y = ring.gemm(ch, sh, dev_u16(NF4), dev_u16(x))
+                outs.append((y, codes, scales, x, ch, sh))
+            torch.cuda.synchronize()
+            for y, codes, scales, x, _, _ in outs:
+                yn = y.cpu().numpy()
+                if M == 1:
+                    assert np.array_equal(yn, run_matmul(codes, scales, NF4, x, "gemv"))
+                assert_close(yn, codes, scales, NF4, x, label=f"ring M={M} N={codes.shape[0]}")
+        # a matrix larger than a slot is refused before anything runs
+        codes, scales = random_packed(99, 2048, 4096)
+        with pytest.raises(q4.Q4Error) as err:
+            ring.gemm(torch.from_numpy(codes), torch.from_numpy(scales.view(np.int16)), dev_u16(NF4),
+                      dev_u16(synth.activations(1, 1, 4096)))
+        assert err.value.status == 6
+    finally:
+        ring.close()
+
+
 def test_no_bounded_wait_ran_out():
     """Collected last in this file: no kernel above gave up on a wait."""
     assert q4.timeout_flags() == 0

@@ -72,6 +72,12 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.q4_abi_version.restype = ctypes.c_int
     lib.q4_timeout_flags.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     lib.q4_timeout_flags.restype = ctypes.c_int
+    lib.q4_ring_create.argtypes = [I64, ctypes.POINTER(ctypes.c_void_p)]
+    lib.q4_ring_create.restype = ctypes.c_int
+    lib.q4_ring_gemm.argtypes = [P, P, P, P, P, P, I64, I64, I64, S]
+    lib.q4_ring_gemm.restype = ctypes.c_int
+    lib.q4_ring_destroy.argtypes = [P]
+    lib.q4_ring_destroy.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -218,6 +224,61 @@ def q4_gemm_noalloc(codes, scales, codebook, x, y, stream=None) -> torch.Tensor:
     if y is None:
         raise ValueError("q4_gemm_noalloc writes into a caller-provided y")
     return _matmul("q4_gemm_noalloc", codes, scales, codebook, x, y, stream)
+
+
+def ring_slot_bytes(N: int, K: int) -> int:
+    """Bytes a CopyRing slot needs for one [N, K] matrix (codes padded to 256
+    bytes, then scales)."""
+    return (N * (K // 2) + 255) // 256 * 256 + N * (K // GROUP) * 2
+
+
+class Ring:
+    """Two device slots fed from host memory ("CopyRing"): ``gemm`` copies a
+    matrix's packed codes and scales from (pinned) host tensors into the next
+    slot on the ring's copy stream and runs q4_gemm on it, so that the copy of
+    one call overlaps the matmul of the previous one."""
+
+    def __init__(self, slot_bytes: int):
+        self._h = ctypes.c_void_p()
+        _check(load().q4_ring_create(int(slot_bytes), ctypes.byref(self._h)), "q4_ring_create")
+
+    def gemm(self, codes_host: torch.Tensor, scales_host: torch.Tensor, codebook: torch.Tensor,
+             x: torch.Tensor, y: torch.Tensor = None, stream=None) -> torch.Tensor:
+        if self._h.value is None:
+            raise RuntimeError("ring is closed")
+        if codes_host.dim() != 2:
+            raise ValueError("codes must be [N, K/2]")
+        N, K = codes_host.shape[0], codes_host.shape[1] * 2
+        for t, name in ((codes_host, "codes_host"), (scales_host, "scales_host")):
+            if t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous host tensor")
+        if codes_host.dtype != torch.uint8 or scales_host.dtype not in _H16 or \
+                tuple(scales_host.shape) != (N, K // GROUP):
+            raise TypeError("codes_host uint8 [N, K/2], scales_host binary16 [N, K/64]")
+        if x.dim() != 2 or x.shape[1] != K:
+            raise ValueError(f"x must be [M, {K}]")
+        M = x.shape[0]
+        if y is None:
+            y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+        _need(codebook, "codebook", _H16, (16,))
+        _need(x, "x", _BF16)
+        _need(y, "y", (torch.float32,), (M, N))
+        st = load().q4_ring_gemm(self._h, codes_host.data_ptr(), scales_host.data_ptr(),
+                                 codebook.data_ptr(), x.data_ptr(), y.data_ptr(), M, N, K,
+                                 _stream(x, stream))
+        _check(st, "q4_ring_gemm")
+        return y
+
+    def close(self) -> None:
+        if self._h.value is not None:
+            _check(load().q4_ring_destroy(self._h), "q4_ring_destroy")
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def timeout_flags() -> int:

@@ -73,6 +73,22 @@ q4_status check_matmul(const uint8_t* codes, const uint16_t* scales, const uint1
     return Q4_OK;
 }
 
+// q4_gemm's kernel choice, after validation.
+q4_status gemm_dispatch(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                        const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
+                        cudaStream_t stream, const DeviceInfo& dev) {
+    if (M <= 16)
+        return after_launch(launch_small_m(codes, scales, cb, x, y, static_cast<int>(M), N, K, stream, dev));
+    if (M <= 24) {
+        // still weight-streaming: the CUDA-core decode kernel beats the
+        // tensor-core pipeline up to 24 tokens (measured crossover on B200)
+        cudaError_t e = launch_gemm_small(codes, scales, cb, x, y, static_cast<int>(M), N, K, stream, dev);
+        if (e != cudaErrorNotSupported) return after_launch(e);
+        (void)cudaGetLastError();
+    }
+    return after_launch(launch_prefill(codes, scales, cb, x, y, M, N, K, stream, dev));
+}
+
 }  // namespace
 
 cudaError_t current_device_info(DeviceInfo* info) {
@@ -117,6 +133,19 @@ cudaError_t ensure_smem_attr(const void* func, int bytes, int slot, int device) 
 }  // namespace q4
 
 using namespace q4;
+
+// Two device slots fed from host memory (see q4_ring_create in q4.h).
+struct q4_ring {
+    std::mutex mu;
+    int device = 0;
+    int64_t slot_bytes = 0;
+    void* slot[2] = {nullptr, nullptr};
+    cudaStream_t copy = nullptr;
+    cudaEvent_t copied[2] = {nullptr, nullptr};  // slot s holds the weights of its latest call
+    cudaEvent_t used[2] = {nullptr, nullptr};    // the matmul that last read slot s is done
+    int next = 0;
+};
+
 
 extern "C" {
 
@@ -184,18 +213,7 @@ q4_status q4_gemm(const uint8_t* codes, const uint16_t* scales, const uint16_t* 
     if (st != Q4_OK || empty) return st;
     DeviceInfo dev;
     if ((st = gate(&dev)) != Q4_OK) return st;
-    if (M <= 16)
-        return after_launch(
-            launch_small_m(codes, scales, codebook, x, y, static_cast<int>(M), N, K, stream, dev));
-    if (M <= 24) {
-        // still weight-streaming: the CUDA-core decode kernel beats the
-        // tensor-core pipeline up to 24 tokens (measured crossover on B200)
-        cudaError_t e = launch_gemm_small(codes, scales, codebook, x, y, static_cast<int>(M), N, K,
-                                          stream, dev);
-        if (e != cudaErrorNotSupported) return after_launch(e);
-        (void)cudaGetLastError();
-    }
-    return after_launch(launch_prefill(codes, scales, codebook, x, y, M, N, K, stream, dev));
+    return gemm_dispatch(codes, scales, codebook, x, y, M, N, K, stream, dev);
 }
 
 q4_status q4_gemm_noalloc(const uint8_t* codes, const uint16_t* scales, const uint16_t* codebook,
@@ -219,6 +237,97 @@ q4_status q4_gemm_noalloc(const uint8_t* codes, const uint16_t* scales, const ui
         (void)cudaGetLastError();
     }
     return after_launch(launch_prefill_noalloc(codes, scales, codebook, x, y, M, N, K, stream, dev));
+}
+
+// Offset of the scales in a slot: after the codes, rounded up to 256 bytes.
+static int64_t ring_scales_offset(int64_t N, int64_t K) { return (N * (K / 2) + 255) / 256 * 256; }
+
+static void ring_free(q4_ring* r) {
+    for (int s = 0; s < 2; ++s) {
+        if (r->slot[s]) cudaFree(r->slot[s]);
+        if (r->copied[s]) cudaEventDestroy(r->copied[s]);
+        if (r->used[s]) cudaEventDestroy(r->used[s]);
+    }
+    if (r->copy) cudaStreamDestroy(r->copy);
+    delete r;
+}
+
+q4_status q4_ring_create(int64_t slot_bytes, q4_ring** ring) {
+    if (!ring) return Q4_ERR_NULL;
+    *ring = nullptr;
+    if (slot_bytes <= 0) return Q4_ERR_SHAPE;
+    DeviceInfo dev;
+    q4_status st = gate(&dev);
+    if (st != Q4_OK) return st;
+    q4_ring* r = new q4_ring();
+    r->device = dev.device;
+    r->slot_bytes = slot_bytes;
+    cudaError_t e = cudaSuccess;
+    for (int s = 0; s < 2 && e == cudaSuccess; ++s) {
+        e = cudaMalloc(&r->slot[s], static_cast<size_t>(slot_bytes));
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r->copied[s], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&r->used[s], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&r->copy, cudaStreamNonBlocking);
+    if (e != cudaSuccess) {
+        ring_free(r);
+        return cuda_fail(e);
+    }
+    *ring = r;
+    return Q4_OK;
+}
+
+q4_status q4_ring_destroy(q4_ring* ring) {
+    if (!ring) return Q4_ERR_NULL;
+    int cur = -1;
+    cudaError_t e = cudaGetDevice(&cur);
+    bool switched = false;
+    if (e == cudaSuccess && cur != ring->device) {
+        e = cudaSetDevice(ring->device);
+        switched = e == cudaSuccess;
+    }
+    // wait for the ring's copies and for the matmuls that read its slots
+    if (e == cudaSuccess) e = cudaStreamSynchronize(ring->copy);
+    for (int s = 0; s < 2 && e == cudaSuccess; ++s) e = cudaEventSynchronize(ring->used[s]);
+    ring_free(ring);
+    if (switched) cudaSetDevice(cur);
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
+}
+
+q4_status q4_ring_gemm(q4_ring* ring, const uint8_t* host_codes, const uint16_t* host_scales,
+                       const uint16_t* codebook, const uint16_t* x, float* y, int64_t M, int64_t N,
+                       int64_t K, q4_stream_t stream) {
+    if (!ring) return Q4_ERR_NULL;
+    bool empty;
+    q4_status st = check_matmul(host_codes, host_scales, codebook, x, y, M, N, K, &empty);
+    if (st != Q4_OK || empty) return st;
+    const int64_t soff = ring_scales_offset(N, K);
+    if (soff + N * (K / kGroup) * 2 > ring->slot_bytes) return Q4_ERR_TOO_LARGE;
+    DeviceInfo dev;
+    if ((st = gate(&dev)) != Q4_OK) return st;
+    if (dev.device != ring->device) return cuda_fail(cudaErrorInvalidDevice);
+    std::lock_guard<std::mutex> lock(ring->mu);
+    const int s = ring->next;
+    uint8_t* dcodes = static_cast<uint8_t*>(ring->slot[s]);
+    uint16_t* dscales = reinterpret_cast<uint16_t*>(dcodes + soff);
+    // the copy waits for the matmul that last read this slot
+    cudaError_t e = cudaStreamWaitEvent(ring->copy, ring->used[s], 0);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(dcodes, host_codes, static_cast<size_t>(N * (K / 2)), cudaMemcpyHostToDevice,
+                            ring->copy);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(dscales, host_scales, static_cast<size_t>(N * (K / kGroup) * 2),
+                            cudaMemcpyHostToDevice, ring->copy);
+    if (e == cudaSuccess) e = cudaEventRecord(ring->copied[s], ring->copy);
+    // the matmul waits for the copy
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, ring->copied[s], 0);
+    if (e != cudaSuccess) return cuda_fail(e);
+    st = gemm_dispatch(dcodes, dscales, codebook, x, y, M, N, K, stream, dev);
+    if (st != Q4_OK) return st;
+    e = cudaEventRecord(ring->used[s], stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    ring->next = s ^ 1;
+    return Q4_OK;
 }
 
 const char* q4_status_string(q4_status status) {
