@@ -688,8 +688,8 @@ def bench_ring(dev, cb, stream, lins, steps=20):
         c0.record()
         for _ in range(5):
             for ch, sh in host:
-                dst[:ch.numel()].copy_(ch, non_blocking=True)
-                dst[:sh.numel() * 2].view(torch.int16).copy_(sh.view(torch.int16), non_blocking=True)
+                dst[:ch.numel()].copy_(ch.view(-1), non_blocking=True)
+                dst[:sh.numel() * 2].view(torch.int16).copy_(sh.view(torch.int16).view(-1), non_blocking=True)
         c1.record()
     c1.synchronize()
     copy_ms = c0.elapsed_time(c1) / 5
