@@ -27,16 +27,19 @@
  *   w        float    [N][K]     binary32 (input of q4_pack, output of q4_dequant)
  *
  * Ownership.  Every pointer is device memory owned by the caller (PyTorch,
- * cudaMalloc, ...).  The library keeps no pointer after a call returns and
- * holds only a per-device cache of the device's properties.  The one
- * allocation it makes is the stream-ordered scratch of the tensor-core path
- * of q4_gemm (M > 24; M = 17..24 only when the M <= 24 kernel declines a
- * shape: 2 * M * K bytes for the binary16 copy of x), taken from a memory pool the
- * library creates once per device and returned to that pool on the same
- * stream before the call returns; the pool keeps the memory it has mapped.
+ * cudaMalloc, ...), except the host-side weights of q4_ring_gemm.  The
+ * library keeps no pointer after a call returns and holds only a per-device
+ * cache of the device's properties.  It allocates in two places: the
+ * stream-ordered scratch of the tensor-core path of q4_gemm (M > 24; M =
+ * 17..24 only when the M <= 24 kernel declines a shape: 2 * M * K bytes for
+ * the binary16 copy of x), taken from a memory pool the library creates once
+ * per device and returned to that pool on the same stream before the call
+ * returns (the pool keeps the memory it has mapped); and the two device slots
+ * of a q4_ring, which the caller creates and destroys explicitly.
  * All calls are asynchronous on the caller's stream (0 = legacy default
- * stream); none synchronizes the host.  Inputs and outputs must not overlap.
- * The calls are thread-safe.
+ * stream); none synchronizes the host except q4_timeout_flags and
+ * q4_ring_destroy.  Inputs and outputs must not overlap.  The calls are
+ * thread-safe.
  *
  * Errors.  Each call validates its arguments before launching anything, in
  * this order, and returns the first failure:
