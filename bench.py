@@ -142,21 +142,34 @@ def setup_dist():
 
 
 def barrier(world):
+    """Every rank reaches this point, and this rank's GPU work is done."""
     import torch
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(v, world):
+    """The largest of the ranks' values (device time: the slowest rank sets the
+    step).  The tensor lives where the process group's backend works: on the
+    GPU for NCCL, on the host for gloo."""
     import torch
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate(units_per_rank, ms_per_step, world):
+    """Whole-job throughput of independent replicas (weak scaling): every rank
+    processes ``units_per_rank`` per step, and the step takes the slowest
+    rank's time."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -367,7 +380,7 @@ def run_ours(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(lins, cb, args.cpu_seconds)
 
-    value = world * bytes_step / (ms_step * 1e-3) / 1e9
+    value = aggregate(bytes_step, ms_step, world) / 1e9
     line = {
         "metric": "q4_gemv HBM GB/s (% of B200 peak) at M=1; q4_gemm TFLOP/s at M>=16",
         "value": round(value, 2),
@@ -406,7 +419,7 @@ def run_ours(args, world, rank, local):
             "timing": f"{COPIES} back-to-back launches in one CUDA graph over rotating weight copies",
         },
         "e2e": {
-            "value": round(world * bytes_step / (e2e_ms * 1e-3) / 1e9, 2),
+            "value": round(aggregate(bytes_step, e2e_ms, world) / 1e9, 2),
             "unit": "GB/s",
             "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h,
