@@ -102,6 +102,14 @@ class Oracle:
         lib.oracle_matmul.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P, P]
         lib.oracle_embed_rows.restype = ctypes.c_int
         lib.oracle_embed_rows.argtypes = [P, P, P, P, I64, I64, I64, P]
+        lib.oracle_pack2.restype = ctypes.c_int
+        lib.oracle_pack2.argtypes = [P, P, P, P, I64, I64]
+        lib.oracle_weight2.restype = ctypes.c_float
+        lib.oracle_weight2.argtypes = [P, P, P, I64, I64, I64]
+        lib.oracle_dequant2.restype = ctypes.c_int
+        lib.oracle_dequant2.argtypes = [P, P, P, P, I64, I64]
+        lib.oracle_matmul2.restype = ctypes.c_int
+        lib.oracle_matmul2.argtypes = [P, P, P, P, I64, I64, I64, P, P]
         self.lib = lib
         self.path = path
 
@@ -172,6 +180,43 @@ class Oracle:
             raise ValueError("oracle_embed_rows: bad shape")
         return out
 
+    # ---- the two-bit variant: cb4 uint16 [4], codes uint8 [N, K/4] ------------
+    def pack2(self, w, cb4):
+        w, cb4 = _c(w, np.float32), _c(cb4, np.uint16)
+        N, K = w.shape
+        codes = np.empty((N, K // 4), np.uint8)
+        scales = np.empty((N, K // GROUP), np.uint16)
+        if self.lib.oracle_pack2(_ptr(w), _ptr(cb4), _ptr(codes), _ptr(scales), N, K) != 0:
+            raise ValueError(f"oracle_pack2: bad shape N={N} K={K}")
+        return codes, scales
+
+    def weight2(self, codes, scales, cb4, n: int, k: int) -> float:
+        codes, scales, cb4 = _c(codes, np.uint8), _c(scales, np.uint16), _c(cb4, np.uint16)
+        return float(self.lib.oracle_weight2(_ptr(codes), _ptr(scales), _ptr(cb4),
+                                             codes.shape[1] * 4, n, k))
+
+    def dequant2(self, codes, scales, cb4) -> np.ndarray:
+        codes, scales, cb4 = _c(codes, np.uint8), _c(scales, np.uint16), _c(cb4, np.uint16)
+        N, K = codes.shape[0], codes.shape[1] * 4
+        out = np.empty((N, K), np.float32)
+        if self.lib.oracle_dequant2(_ptr(codes), _ptr(scales), _ptr(cb4), _ptr(out), N, K) != 0:
+            raise ValueError("oracle_dequant2: bad shape")
+        return out
+
+    def matmul2(self, codes, scales, cb4, x):
+        codes, scales, cb4 = _c(codes, np.uint8), _c(scales, np.uint16), _c(cb4, np.uint16)
+        x = _c(x, np.uint16)
+        N, K = codes.shape[0], codes.shape[1] * 4
+        M = x.shape[0]
+        if x.shape[1] != K:
+            raise ValueError("x has the wrong K")
+        y = np.empty((M, N), np.float32)
+        a = np.empty((M, N), np.float64)
+        if self.lib.oracle_matmul2(_ptr(codes), _ptr(scales), _ptr(cb4), _ptr(x), M, N, K,
+                                   _ptr(y), _ptr(a)) != 0:
+            raise ValueError("oracle_matmul2: bad arguments")
+        return y, a
+
     def matmul(self, codes, scales, cb, x, rows=None, with_abs: bool = True):
         """y [M, n_out] (fp32) and sum|W*x| [M, n_out] (fp64, or None).
 
@@ -217,3 +262,7 @@ def dequant(codes, scales, cb): return default().dequant(codes, scales, cb)
 def matmul(codes, scales, cb, x, rows=None, with_abs=True):
     return default().matmul(codes, scales, cb, x, rows, with_abs)
 def embed_rows(codes, scales, cb, ids): return default().embed_rows(codes, scales, cb, ids)
+def pack2(w, cb4): return default().pack2(w, cb4)
+def weight2(codes, scales, cb4, n, k): return default().weight2(codes, scales, cb4, n, k)
+def dequant2(codes, scales, cb4): return default().dequant2(codes, scales, cb4)
+def matmul2(codes, scales, cb4, x): return default().matmul2(codes, scales, cb4, x)

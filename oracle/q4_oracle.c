@@ -39,7 +39,9 @@
  *  - matmul reference: the products W * x summed in fp64 in increasing k and
  *    rounded once to binary32;
  *  - embedding rows: the requested rows of the dequantized matrix in binary32;
- *    an id outside [0, N) gives a row of zeros.
+ *    an id outside [0, N) gives a row of zeros;
+ *  - the two-bit variant (the pages name 2-bit codebooks, print none): the same
+ *    steps with a 4-entry codebook and four codes per byte (see below).
  */
 #include "q4_oracle.h"
 
@@ -323,5 +325,117 @@ int oracle_matmul(const uint8_t* codes, const uint16_t* scales,
         }
     }
     free(wrow);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Two-bit variant: a 4-entry codebook, four codes per byte                  */
+/* ------------------------------------------------------------------------ */
+/* "Trapetum" overview, sections "In one sentence" and "Frontier models on
+ * your own hardware": a 70B model in 2 bits; the pages print no 2-bit layout.
+ * Reading: the 4-bit
+ * format with 2-bit codes -- groups of 64 along K and one binary16 scale per
+ * group (binary16 of the group's absmax, rounded to nearest-even); a code is
+ * the index of the entry nearest to w / scale (binary32, ties to the lowest
+ * index); a zero scale gives every weight the entry of smallest magnitude;
+ * byte j of a row holds k = 4j + i in bits 2i and 2i + 1. */
+
+static int nearest_of_four(float q, const float e[4])
+{
+    int pick = 0;
+    float dist = fabsf(q - e[0]);
+    for (int i = 1; i < 4; ++i) {
+        float di = fabsf(q - e[i]);
+        if (di < dist) {
+            dist = di;
+            pick = i;
+        }
+    }
+    return pick;
+}
+
+int oracle_pack2(const float* w, const uint16_t* cb4, uint8_t* codes,
+                 uint16_t* scales, int64_t N, int64_t K)
+{
+    if (N < 0 || K <= 0 || K % ORACLE_GROUP != 0)
+        return -1;
+    float e[4];
+    for (int i = 0; i < 4; ++i)
+        e[i] = oracle_h2f(cb4[i]);
+    int least = 0;
+    for (int i = 1; i < 4; ++i)
+        if (fabsf(e[i]) < fabsf(e[least]))
+            least = i;
+    const int64_t G = K / ORACLE_GROUP;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t g = 0; g < G; ++g) {
+            const float* src = w + n * K + g * ORACLE_GROUP;
+            float amax = 0.0f;
+            for (int j = 0; j < ORACLE_GROUP; ++j) {
+                float t = fabsf(src[j]);
+                if (t > amax)
+                    amax = t;
+            }
+            uint16_t sbits = oracle_f2h_rne(amax);
+            float sv = oracle_h2f(sbits);
+            scales[n * G + g] = sbits;
+            uint8_t* dst = codes + n * (K / 4) + g * (ORACLE_GROUP / 4);
+            for (int j = 0; j < ORACLE_GROUP / 4; ++j)
+                dst[j] = 0;
+            for (int j = 0; j < ORACLE_GROUP; ++j) {
+                int code = (sv == 0.0f) ? least : nearest_of_four(src[j] / sv, e);
+                dst[j / 4] = (uint8_t)(dst[j / 4] | (code << (2 * (j % 4))));
+            }
+        }
+    }
+    return 0;
+}
+
+float oracle_weight2(const uint8_t* codes, const uint16_t* scales,
+                     const uint16_t* cb4, int64_t K, int64_t n, int64_t k)
+{
+    uint8_t b = codes[n * (K / 4) + k / 4];
+    int code = (b >> (2 * (k % 4))) & 3;
+    float val = oracle_h2f(cb4[code]);
+    float sc = oracle_h2f(scales[n * (K / ORACLE_GROUP) + (k / ORACLE_GROUP)]);
+    return val * sc;
+}
+
+int oracle_dequant2(const uint8_t* codes, const uint16_t* scales,
+                    const uint16_t* cb4, float* w_out, int64_t N, int64_t K)
+{
+    if (N < 0 || K <= 0 || K % ORACLE_GROUP != 0)
+        return -1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t kk = 0; kk < K; ++kk)
+            w_out[n * K + kk] = oracle_weight2(codes, scales, cb4, K, n, kk);
+    return 0;
+}
+
+int oracle_matmul2(const uint8_t* codes, const uint16_t* scales,
+                   const uint16_t* cb4, const uint16_t* x, int64_t M,
+                   int64_t N, int64_t K, float* y, double* absacc)
+{
+    if (M < 0 || N < 0 || K <= 0 || K % ORACLE_GROUP != 0)
+        return -1;
+    float* row = (float*)malloc((size_t)K * sizeof(float));
+    if (!row)
+        return -1;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t kk = 0; kk < K; ++kk)
+            row[kk] = oracle_weight2(codes, scales, cb4, K, n, kk);
+        for (int64_t m = 0; m < M; ++m) {
+            double sum = 0.0, abs_sum = 0.0;
+            for (int64_t kk = 0; kk < K; ++kk) {
+                double prod = (double)row[kk] * (double)oracle_bf2f(x[m * K + kk]);
+                sum += prod;
+                abs_sum += fabs(prod);
+            }
+            y[m * N + n] = (float)sum;
+            if (absacc)
+                absacc[m * N + n] = abs_sum;
+        }
+    }
+    free(row);
     return 0;
 }

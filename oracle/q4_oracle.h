@@ -69,4 +69,18 @@ int      oracle_matmul(const uint8_t* codes, const uint16_t* scales,
 #ifdef __cplusplus
 }
 #endif
+/* Two-bit variant (4-entry codebook cb4, codes [N][K/4], byte j holds
+ * k = 4j + i in bits 2i, 2i+1; scales as the 4-bit format): pack, one weight,
+ * dense dequantization, and the fp64 matmul (y [M][N], absacc may be NULL).
+ * Each returns 0 or -1 for a bad shape, except oracle_weight2. */
+int      oracle_pack2(const float* w, const uint16_t* cb4, uint8_t* codes,
+                      uint16_t* scales, int64_t N, int64_t K);
+float    oracle_weight2(const uint8_t* codes, const uint16_t* scales,
+                        const uint16_t* cb4, int64_t K, int64_t n, int64_t k);
+int      oracle_dequant2(const uint8_t* codes, const uint16_t* scales,
+                         const uint16_t* cb4, float* w_out, int64_t N, int64_t K);
+int      oracle_matmul2(const uint8_t* codes, const uint16_t* scales,
+                        const uint16_t* cb4, const uint16_t* x, int64_t M,
+                        int64_t N, int64_t K, float* y, double* absacc);
+
 #endif

@@ -117,6 +117,12 @@ def tiny_codes_scales(seed: int, N: int, K: int):
     return codes, scales
 
 
+def codebook2() -> np.ndarray:
+    """A synthetic 4-entry codebook for the two-bit variant, as binary16 bit
+    patterns: -1, -1/3, 1/3, 1 (each rounded to binary16)."""
+    return np.array([-1.0, -1.0 / 3.0, 1.0 / 3.0, 1.0], dtype=np.float16).view(np.uint16)
+
+
 def codebook() -> np.ndarray:
     """The NF4 codebook as 16 binary16 bit patterns, read from the committed fixture."""
     vals = []

@@ -389,6 +389,106 @@ def pin_embed_rows_definition(o):
         assert np.array_equal(got[i], want), f"row {i} (id {n})"
 
 
+# ---- the two-bit variant (4-entry codebook, four codes per byte) -----------
+
+CB4 = synth.codebook2()
+
+
+def _decode2_numpy(codes, scales, cb4):
+    """W of the two-bit format straight from the bytes, with numpy's own
+    binary16 -> binary32 conversion and binary32 product."""
+    N, K = codes.shape[0], codes.shape[1] * 4
+    cbf = cb4.view(np.float16).astype(np.float32)
+    sf = scales.view(np.float16).astype(np.float32)
+    idx = np.empty((N, K), np.uint8)
+    for i in range(4):
+        idx[:, i::4] = (codes >> (2 * i)) & 3
+    return cbf[idx] * np.repeat(sf, GROUP, axis=1)
+
+
+def pin_two_bit_bit_order(o):
+    """Byte 0xE4 = 0b11_10_01_00 holds codes 0, 1, 2, 3 for k = 0..3."""
+    codes = np.full((1, GROUP // 4), 0xE4, np.uint8)
+    scales = np.array([[0x3C00]], np.uint16)                 # scale 1
+    cbf = CB4.view(np.float16).astype(np.float32)
+    for k in range(4):
+        assert o.weight2(codes, scales, CB4, 0, k) == cbf[k]
+
+
+def pin_two_bit_dequant_definition(o):
+    rng = np.random.default_rng(21)
+    N, K = 9, 3 * GROUP
+    codes = rng.integers(0, 256, size=(N, K // 4), dtype=np.uint8)
+    scales = synth.f32_to_f16_bits(rng.uniform(0.005, 0.05, size=(N, K // GROUP)).astype(np.float32))
+    assert np.array_equal(o.dequant2(codes, scales, CB4), _decode2_numpy(codes, scales, CB4))
+
+
+def pin_two_bit_pack_round_trip(o):
+    """W built on the grid (each group holds a code of magnitude 1, so the
+    absmax is the scale) packs back to the same codes and scales."""
+    rng = np.random.default_rng(22)
+    N, K = 6, 4 * GROUP
+    idx = rng.integers(0, 4, size=(N, K)).astype(np.uint8)
+    idx[:, ::GROUP] = 3                                       # cb4[3] = +1 in every group
+    s = np.asarray(2.0 ** rng.integers(-8, -3, size=(N, K // GROUP)), np.float16)
+    w = CB4.view(np.float16).astype(np.float32)[idx] * np.repeat(s.astype(np.float32), GROUP, axis=1)
+    codes, scales = o.pack2(w, CB4)
+    assert np.array_equal(scales, s.view(np.uint16))
+    assert np.array_equal(_decode2_numpy(codes, scales, CB4), w)
+
+
+def pin_two_bit_pack_brute_force(o):
+    """Each code is the nearest entry to w / scale in binary32, ties to the
+    lowest index; scale = binary16(absmax); zero groups take the entry of
+    smallest magnitude (index 1: |-1/3| ties |1/3|, lowest index)."""
+    rng = np.random.default_rng(23)
+    N, K = 7, 2 * GROUP
+    w = (rng.standard_normal((N, K)) * 0.03).astype(np.float32)
+    w[2, :GROUP] = 0.0
+    codes, scales = o.pack2(w, CB4)
+    cbf = CB4.view(np.float16).astype(np.float32)
+    amax = np.abs(w.reshape(N, K // GROUP, GROUP)).max(axis=2)
+    assert np.array_equal(scales, amax.astype(np.float16).view(np.uint16))
+    sf = np.repeat(scales.view(np.float16).astype(np.float32), GROUP, axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r = (w / sf).astype(np.float32)
+    want = np.argmin(np.abs(r[..., None] - cbf), axis=-1)
+    want[sf == 0] = 1
+    got = np.empty((N, K), np.int64)
+    for i in range(4):
+        got[:, i::4] = (codes >> (2 * i)) & 3
+    assert np.array_equal(got, want)
+
+
+def pin_two_bit_pack_ties(o):
+    """Values exactly halfway between two entries take the lower index:
+    0 sits between -1/3 and 1/3 (index 1), the midpoints of the binary16
+    entries (exact in binary32) go to indices 0, 1 and 2."""
+    cbf = CB4.view(np.float16).astype(np.float32)
+    mids = [(cbf[0] + cbf[1]) / 2, np.float32(0.0), (cbf[2] + cbf[3]) / 2]
+    w = np.zeros((1, GROUP), np.float32)
+    w[0, 0] = 0.25                                            # absmax, a power of two
+    w[0, 1:4] = np.array(mids, np.float32) * np.float32(0.25)
+    codes, scales = o.pack2(w, CB4)
+    assert scales[0, 0] == 0x3400
+    got = [(codes[0, k // 4] >> (2 * (k % 4))) & 3 for k in range(4)]
+    assert got == [3, 0, 1, 2]
+
+
+def pin_two_bit_matmul_brute_force(o):
+    rng = np.random.default_rng(24)
+    N, K, M = 11, 2 * GROUP, 3
+    codes = rng.integers(0, 256, size=(N, K // 4), dtype=np.uint8)
+    scales = synth.f32_to_f16_bits(rng.uniform(0.005, 0.05, size=(N, K // GROUP)).astype(np.float32))
+    x = synth.f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    y, a = o.matmul2(codes, scales, CB4, x)
+    W = _decode2_numpy(codes, scales, CB4).astype(np.float64)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    ref = np.array([[sum(W[n, k] * xf[m, k] for k in range(K)) for n in range(N)] for m in range(M)])
+    assert np.array_equal(y, ref.astype(np.float32))
+    assert np.allclose(a, np.abs(xf) @ np.abs(W).T, rtol=1e-13, atol=0)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
 
 
@@ -456,6 +556,12 @@ MUTANTS = {
                                    "oracle_weight(codes, scales, cb, K, n < 0 ? 0 : (n >= N ? N - 1 : n), k)"),
     "embed_row_off_by_one": ("? oracle_weight(codes, scales, cb, K, n, k)",
                              "? oracle_weight(codes, scales, cb, K, n > 0 ? n - 1 : 0, k)"),
+    "two_bit_order_reversed": ("int code = (b >> (2 * (k % 4))) & 3;", "int code = (b >> (2 * (3 - k % 4))) & 3;"),
+    "two_bit_pack_order_reversed": ("(code << (2 * (j % 4)))", "(code << (2 * (3 - j % 4)))"),
+    "two_bit_tie_to_highest": ("if (di < dist) {", "if (di <= dist) {"),
+    "two_bit_scale_wrong_group": ("+ (k / ORACLE_GROUP)]);", "+ (k / ORACLE_GROUP) / 2]);"),
+    "two_bit_zero_scale_first": ("(sv == 0.0f) ? least :", "(sv == 0.0f) ? 0 :"),
+    "two_bit_abs_sum_signed": ("abs_sum += fabs(prod);", "abs_sum += prod;"),
 }
 
 
