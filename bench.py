@@ -374,6 +374,7 @@ def run_ours(args, world, rank, local):
     smallm = None if args.no_smallm else bench_small_m(dev, cb, stream, hbm_peak)
     embed = None if args.no_smallm else bench_embed_rows(dev, cb, stream, hbm_peak)
     ring = None if args.no_smallm else bench_ring(dev, cb, stream, lins)
+    two_bit = None if args.no_smallm else bench_gemv2(dev, stream, hbm_peak)
 
     # ---- CPU baseline: the oracle on the host --------------------------------
     cpu = None
@@ -442,6 +443,8 @@ def run_ours(args, world, rank, local):
         line["embed_rows"] = embed
     if ring is not None:
         line["copy_ring"] = ring
+    if two_bit is not None:
+        line["two_bit_gemv_llama2_70b"] = two_bit
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if rank == 0:
@@ -663,6 +666,69 @@ def bench_embed_rows(dev, cb, stream, hbm_peak, n_ids=4096, reps=20):
             "us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
             "hbm_frac_of_measured": round(gbs / hbm_peak, 4),
             "timing": "CUDA graph of 4 calls on different ids, replayed 20 times"}
+
+
+def bench_gemv2(dev, stream, hbm_peak, reps=20):
+    """The two-bit variant: the Llama-2-70B decoder layer's four linears at
+    M = 1 (q4_gemv2; uniform random 2-bit codes and U[0.005, 0.05] scales,
+    241 MB per layer, more than L2), one CUDA graph of the four calls."""
+    import torch
+    import weight_only_bit_gemv_b200 as q4
+    cb4 = torch.from_numpy(synth.codebook2().view(np.int16)).to(dev)
+    lins = []
+    for lin in synth.WORKLOADS["llama2_70b_prefill"].linears:
+        g = torch.Generator(device=dev)
+        g.manual_seed(synth.seed_for(5, 0, lin.name))
+        codes = torch.randint(0, 256, (lin.N, lin.K // 4), generator=g, device=dev, dtype=torch.uint8)
+        scales = (torch.rand((lin.N, lin.K // GROUP), generator=g, device=dev) * 0.045 + 0.005).half()
+        x = synth.activations_device(synth.x_seed(synth.seed_for(5, 0, lin.name)), 1, lin.K, dev)
+        y = torch.empty((1, lin.N), dtype=torch.float32, device=dev)
+        lins.append((lin, codes, scales, x, y))
+    with torch.cuda.stream(stream):
+        for lin, c, sc, x, y in lins:
+            q4.q4_gemv2(c, sc, cb4, x, y)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for lin, c, sc, x, y in lins:
+            q4.q4_gemv2(c, sc, cb4, x, y)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            graph.replay()
+        e0.record()
+        for _ in range(reps):
+            graph.replay()
+        e1.record()
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    # algorithmic bytes: codes, scales, x and y of each linear, the codebook
+    nbytes = sum(l.N * l.K // 4 + l.N * (l.K // GROUP) * 2 + 2 * l.K + 4 * l.N + 8 for l, *_ in lins)
+    per = {}
+    for lin, c, sc, x, y in lins:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            t0.record()
+            for _ in range(reps):
+                q4.q4_gemv2(c, sc, cb4, x, y)
+            t1.record()
+        t1.synchronize()
+        us = t0.elapsed_time(t1) * 1e3 / reps
+        b = lin.N * lin.K // 4 + lin.N * (lin.K // GROUP) * 2 + 2 * lin.K + 4 * lin.N + 8
+        per[lin.name] = {"N": lin.N, "K": lin.K, "us": round(us, 2),
+                         "gbs": round(b / (us * 1e-6) / 1e9, 1)}
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    del graph, lins
+    torch.cuda.empty_cache()
+    return {"workload": "llama2_70b decoder layer in 2 bits (4-entry codebook), M=1, "
+                        "4 q4_gemv2 calls (qkv 8192->10240, o, gate_up 8192->57344, down)",
+            "us_per_layer": round(ms * 1e3, 2), "gbs": round(gbs, 1),
+            "hbm_frac_of_measured": round(gbs / hbm_peak, 4), "bytes_per_layer": nbytes,
+            "per_linear_back_to_back": per,
+            "timing": "CUDA graph of the 4 calls (each a y memset and one kernel), replayed 20 times; "
+                      "per linear: 20 back-to-back calls"}
 
 
 def bench_ring(dev, cb, stream, lins, steps=20):

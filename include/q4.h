@@ -268,6 +268,38 @@ int q4_last_cuda_error(void);
 int q4_abi_version(void);
 
 /*
+ * The two-bit variant: the same groups of 64 weights and binary16 scales,
+ * 2-bit codes into a 4-entry binary16 codebook.
+ * Source: "Trapetum" overview, "In one sentence" and "Frontier models on your
+ * own hardware" (a 70B model in 2 bits on one 24 GB card).  The pages print
+ * no 2-bit layout; this one is the 4-bit layout with four codes per byte:
+ *   codes     uint8_t  [N][K/4]   byte j of row n holds code(n, 4j + i) in
+ *                                 bits 2i and 2i + 1 (i = 0..3)
+ *   scales    uint16_t [N][K/64]  binary16 bit patterns
+ *   codebook4 uint16_t [4]        binary16 bit patterns (any values, any order)
+ *   W[n][k] = codebook4[code(n, k)] * scale[n][k / 64]
+ *
+ * q4_pack2 / q4_dequant2: q4_pack / q4_dequant with 4 entries (nearest entry
+ * in binary32, ties to the lowest index; a zero scale gives the entry of
+ * smallest magnitude); bit-identical to a serial IEEE implementation.
+ * q4_gemv2: one token, y[n] = sum_k W[n][k] * x[k], x [K] bfloat16, y [N]
+ * fp32.  Products are exact (x rounded to binary16, as q4_gemv), the sums
+ * fp32.  y is zeroed on the stream and then accumulated by several CTAs, so
+ * the order of the fp32 additions is not fixed from run to run.
+ * Validation as q4_dequant / q4_gemv (M = 1 implied), plus Q4_ERR_SHAPE for
+ * K > Q4_GEMV2_MAX_K (x is staged in shared memory, 136 bytes per group).
+ */
+#define Q4_GEMV2_MAX_K 98304
+q4_status q4_pack2(const float* w, const uint16_t* codebook4, uint8_t* codes,
+                   uint16_t* scales, int64_t N, int64_t K, q4_stream_t stream);
+q4_status q4_dequant2(const uint8_t* codes, const uint16_t* scales,
+                      const uint16_t* codebook4, float* w_out, int64_t N,
+                      int64_t K, q4_stream_t stream);
+q4_status q4_gemv2(const uint8_t* codes, const uint16_t* scales,
+                   const uint16_t* codebook4, const uint16_t* x, float* y,
+                   int64_t N, int64_t K, q4_stream_t stream);
+
+/*
  * q4_timeout_flags -- every wait inside the bulk-copy and tensor-core
  * kernels is bounded (about two seconds); a wait that runs out sets a bit in
  * a device word, the kernel drains what it has in flight, frees its tensor

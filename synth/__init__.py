@@ -117,6 +117,15 @@ def tiny_codes_scales(seed: int, N: int, K: int):
     return codes, scales
 
 
+def tiny_codes2_scales(seed: int, N: int, K: int):
+    """Uniform 2-bit codes (four per byte, every byte value equally likely)
+    and binary16 scales U[0.005, 0.05], for the two-bit variant."""
+    r = _rng(seed)
+    codes = r.integers(0, 256, size=(N, K // 4), dtype=np.uint8)
+    scales = f32_to_f16_bits(r.uniform(0.005, 0.05, size=(N, K // 64)).astype(np.float32))
+    return codes, scales
+
+
 def codebook2() -> np.ndarray:
     """A synthetic 4-entry codebook for the two-bit variant, as binary16 bit
     patterns: -1, -1/3, 1/3, 1 (each rounded to binary16)."""

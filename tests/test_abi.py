@@ -106,6 +106,22 @@ def test_embed_rows_rejects(lib):
     assert f(A, A, A, A, MIS, 4, 64, 64, None) == ALIGN
 
 
+def test_two_bit_rejects(lib):
+    for f in (lib.q4_pack2, lib.q4_dequant2):
+        assert f(A, A, A, A, 4, 100, None) == SHAPE            # K % 64
+        assert f(A, A, A, A, -1, 64, None) == SHAPE            # N < 0
+        assert f(None, None, None, None, 0, 64, None) == OK    # N == 0: no launch
+        assert f(None, A, A, A, 4, 64, None) == NULL
+        assert f(MIS, A, A, A, 4, 64, None) == ALIGN
+    g = lib.q4_gemv2
+    assert g(A, A, A, A, A, 4, 100, None) == SHAPE              # K % 64
+    assert g(A, A, A, A, A, 4, 98304 + 64, None) == SHAPE       # above Q4_GEMV2_MAX_K
+    assert g(A, A, A, A, A, -1, 64, None) == SHAPE
+    assert g(None, None, None, None, None, 0, 64, None) == OK   # N == 0: no launch
+    assert g(A, A, A, None, A, 4, 64, None) == NULL
+    assert g(A, A, A, A, MIS, 4, 64, None) == ALIGN
+
+
 def test_ring_rejects(lib):
     import ctypes
     h = ctypes.c_void_p()

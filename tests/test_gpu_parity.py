@@ -107,6 +107,93 @@ def test_embed_rows_bit_exact(N, K, n_ids):
     assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))
 
 
+# ---------------------------------------------------------------------------
+# the two-bit variant (4-entry codebook, four codes per byte)
+# ---------------------------------------------------------------------------
+
+CB4 = synth.codebook2()
+
+
+@pytest.mark.parametrize("N,K", [(128, 256), (1, 64), (37, 448), (300, 4096)])
+def test_pack2_dequant2_bit_exact(N, K):
+    w = synth.weights(77 + N, N, K, 0.02)
+    w[0, :GROUP] = 0.0                                  # a zero group
+    c_ref, s_ref = oracle.pack2(w, CB4)
+    c, s = q4.q4_pack2(torch.from_numpy(w).cuda(), dev_u16(CB4))
+    torch.cuda.synchronize()
+    assert np.array_equal(s.cpu().numpy().view(np.uint16), s_ref)
+    assert np.array_equal(c.cpu().numpy(), c_ref)
+    wd = q4.q4_dequant2(dev_u8(c_ref), dev_u16(s_ref), dev_u16(CB4))
+    torch.cuda.synchronize()
+    assert np.array_equal(wd.cpu().numpy().view(np.uint32), oracle.dequant2(c_ref, s_ref, CB4).view(np.uint32))
+
+
+def test_pack2_ties_on_gpu():
+    """Values halfway between two entries (exact in binary32) take the lower index."""
+    cbf = CB4.view(np.float16).astype(np.float32)
+    w = np.zeros((3, 2 * GROUP), np.float32)
+    w[:, 0] = 0.25
+    w[:, 1:4] = np.array([(cbf[0] + cbf[1]) / 2, 0.0, (cbf[2] + cbf[3]) / 2], np.float32) * np.float32(0.25)
+    w[1, GROUP:] = -0.5                                 # all equal: every code is index 0
+    c_ref, s_ref = oracle.pack2(w, CB4)
+    c, s = q4.q4_pack2(torch.from_numpy(w).cuda(), dev_u16(CB4))
+    torch.cuda.synchronize()
+    assert np.array_equal(c.cpu().numpy(), c_ref) and np.array_equal(s.cpu().numpy().view(np.uint16), s_ref)
+
+
+def run_gemv2(codes, scales, x):
+    y = torch.full((1, codes.shape[0]), float("nan"), dtype=torch.float32, device="cuda")
+    q4.q4_gemv2(dev_u8(codes), dev_u16(scales), dev_u16(CB4), dev_u16(x), y)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+def assert_close2(y, codes, scales, x, label=""):
+    y_ref, a = oracle.matmul2(codes, scales, CB4, x)
+    ok, worst = within_tolerance(y, y_ref, a)
+    assert ok, f"{label}: worst err/bound = {worst:.3g}"
+
+
+# ragged: N not a multiple of 16 (row tiles), K/64 not a multiple of 4
+# (chunks of four groups), and shapes where some warps get no work
+@pytest.mark.parametrize("N,K", [(1, 64), (17, 192), (33, 320), (16, 256), (300, 4096),
+                                 (1000, 1088), (4099, 8192), (5, 98304)])
+def test_gemv2_ragged(N, K):
+    codes, scales = synth.tiny_codes2_scales(900 + N, N, K)
+    x = synth.activations(901 + N, 1, K)
+    assert_close2(run_gemv2(codes, scales, x), codes, scales, x, label=f"{N}x{K}")
+
+
+def test_gemv2_integer_codebook_exact():
+    """Codebook {-2, -1, 1, 2}, power-of-two scales and small-integer x: every
+    partial sum is an integer times a power of two, so y is exact."""
+    cb = np.array([-2.0, -1.0, 1.0, 2.0], np.float16).view(np.uint16)
+    rng = np.random.default_rng(3)
+    N, K = 70, 1024
+    codes = rng.integers(0, 256, size=(N, K // 4), dtype=np.uint8)
+    scales = np.asarray(2.0 ** rng.integers(-4, 2, size=(N, K // GROUP)), np.float16).view(np.uint16)
+    x = synth.f32_to_bf16_bits(rng.integers(-8, 9, size=(1, K)).astype(np.float32))
+    y = torch.full((1, N), float("nan"), dtype=torch.float32, device="cuda")
+    q4.q4_gemv2(dev_u8(codes), dev_u16(scales), dev_u16(cb), dev_u16(x), y)
+    torch.cuda.synchronize()
+    y_ref, _ = oracle.matmul2(codes, scales, cb, x)
+    assert np.array_equal(y.cpu().numpy(), y_ref)
+
+
+@pytest.mark.parametrize("linear", ["qkv", "o", "gate_up", "down"])
+def test_gemv2_llama2_70b_layer(linear):
+    """The Llama-2-70B decoder layer's linears in 2 bits at M = 1: 1024 sampled
+    rows of the full-size launch against the oracle."""
+    lin = {l.name: l for l in synth.WORKLOADS["llama2_70b_prefill"].linears}[linear]
+    seed = synth.seed_for(5, 0, linear)
+    codes, scales = synth.tiny_codes2_scales(seed, lin.N, lin.K)
+    x = synth.activations(synth.x_seed(seed), 1, lin.K)
+    y = run_gemv2(codes, scales, x)
+    rows = np.random.default_rng(seed).choice(lin.N, size=1024, replace=False)
+    rows[:2] = [0, lin.N - 1]
+    assert_close2(y[:, rows], codes[rows], scales[rows], x, label=linear)
+
+
 @pytest.mark.parametrize("N,K", [(128, 256), (1, 64), (37, 448), (300, 4096)])
 def test_pack_dequant_bit_exact(N, K):
     w = synth.weights(7 + N, N, K, 0.02)

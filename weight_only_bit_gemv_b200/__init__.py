@@ -62,7 +62,11 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.q4_gemm.argtypes = [P, P, P, P, P, I64, I64, I64, S]
     lib.q4_gemm_noalloc.argtypes = [P, P, P, P, P, I64, I64, I64, S]
     lib.q4_embed_rows.argtypes = [P, P, P, P, P, I64, I64, I64, S]
-    for f in ("q4_pack", "q4_dequant", "q4_gemv", "q4_gemm", "q4_gemm_noalloc", "q4_embed_rows"):
+    lib.q4_pack2.argtypes = [P, P, P, P, I64, I64, S]
+    lib.q4_dequant2.argtypes = [P, P, P, P, I64, I64, S]
+    lib.q4_gemv2.argtypes = [P, P, P, P, P, I64, I64, S]
+    for f in ("q4_pack", "q4_dequant", "q4_gemv", "q4_gemm", "q4_gemm_noalloc", "q4_embed_rows",
+              "q4_pack2", "q4_dequant2", "q4_gemv2"):
         getattr(lib, f).restype = ctypes.c_int
     lib.q4_status_string.argtypes = [ctypes.c_int]
     lib.q4_status_string.restype = ctypes.c_char_p
@@ -202,6 +206,67 @@ def _matmul(fn: str, codes, scales, codebook, x, y, stream):
     st = getattr(load(), fn)(codes.data_ptr(), scales.data_ptr(), codebook.data_ptr(),
                              x.data_ptr(), y.data_ptr(), M, N, K, _stream(codes, stream))
     _check(st, fn)
+    return y
+
+
+# ---- the two-bit variant: codes [N, K/4], a 4-entry codebook ---------------
+
+def q4_pack2(w: torch.Tensor, codebook4: torch.Tensor, codes: torch.Tensor = None,
+             scales: torch.Tensor = None, stream=None):
+    """Quantize w [N, K] fp32 into 2-bit (codes [N, K/4], scales [N, K/64])."""
+    if w.dim() != 2:
+        raise ValueError("w must be [N, K]")
+    N, K = w.shape
+    if codes is None:
+        codes = torch.empty((N, K // 4), dtype=torch.uint8, device=w.device)
+    if scales is None:
+        scales = torch.empty((N, K // GROUP), dtype=torch.float16, device=w.device)
+    _need(w, "w", (torch.float32,))
+    _need(codebook4, "codebook4", _H16, (4,))
+    _need(codes, "codes", (torch.uint8,), (N, K // 4))
+    _need(scales, "scales", _H16, (N, K // GROUP))
+    st = load().q4_pack2(w.data_ptr(), codebook4.data_ptr(), codes.data_ptr(), scales.data_ptr(),
+                         N, K, _stream(w, stream))
+    _check(st, "q4_pack2")
+    return codes, scales
+
+
+def _packed2_dims(codes: torch.Tensor):
+    if codes.dim() != 2:
+        raise ValueError("codes must be [N, K/4]")
+    return codes.shape[0], codes.shape[1] * 4
+
+
+def q4_dequant2(codes: torch.Tensor, scales: torch.Tensor, codebook4: torch.Tensor,
+                w_out: torch.Tensor = None, stream=None) -> torch.Tensor:
+    N, K = _packed2_dims(codes)
+    if w_out is None:
+        w_out = torch.empty((N, K), dtype=torch.float32, device=codes.device)
+    _need(codes, "codes", (torch.uint8,))
+    _need(scales, "scales", _H16, (N, K // GROUP))
+    _need(codebook4, "codebook4", _H16, (4,))
+    _need(w_out, "w_out", (torch.float32,), (N, K))
+    st = load().q4_dequant2(codes.data_ptr(), scales.data_ptr(), codebook4.data_ptr(),
+                            w_out.data_ptr(), N, K, _stream(codes, stream))
+    _check(st, "q4_dequant2")
+    return w_out
+
+
+def q4_gemv2(codes, scales, codebook4, x, y=None, stream=None) -> torch.Tensor:
+    """y [1, N] = x [1, K] @ W^T with W rebuilt from the 2-bit codes in the kernel."""
+    N, K = _packed2_dims(codes)
+    if x.dim() != 2 or tuple(x.shape) != (1, K):
+        raise ValueError(f"x must be [1, {K}]")
+    if y is None:
+        y = torch.empty((1, N), dtype=torch.float32, device=codes.device)
+    _need(codes, "codes", (torch.uint8,))
+    _need(scales, "scales", _H16, (N, K // GROUP))
+    _need(codebook4, "codebook4", _H16, (4,))
+    _need(x, "x", _BF16)
+    _need(y, "y", (torch.float32,), (1, N))
+    st = load().q4_gemv2(codes.data_ptr(), scales.data_ptr(), codebook4.data_ptr(),
+                         x.data_ptr(), y.data_ptr(), N, K, _stream(codes, stream))
+    _check(st, "q4_gemv2")
     return y
 
 

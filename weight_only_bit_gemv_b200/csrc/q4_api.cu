@@ -348,6 +348,50 @@ int q4_last_cuda_error(void) { return g_last_cuda_error; }
 
 int q4_abi_version(void) { return Q4_ABI_VERSION; }
 
+q4_status q4_pack2(const float* w, const uint16_t* codebook4, uint8_t* codes, uint16_t* scales,
+                   int64_t N, int64_t K, q4_stream_t stream) {
+    q4_status st = check_K(K);
+    if (st != Q4_OK) return st;
+    if (N < 0 || N > Q4_MAX_MN) return Q4_ERR_SHAPE;
+    if (N == 0) return Q4_OK;
+    if (!w || !codebook4 || !codes || !scales) return Q4_ERR_NULL;
+    if (!aligned16(w) || !aligned16(codebook4) || !aligned16(codes) || !aligned16(scales))
+        return Q4_ERR_ALIGN;
+    DeviceInfo dev;
+    if ((st = gate(&dev)) != Q4_OK) return st;
+    return after_launch(launch_pack2(w, codebook4, codes, scales, N, K, stream, dev));
+}
+
+q4_status q4_dequant2(const uint8_t* codes, const uint16_t* scales, const uint16_t* codebook4,
+                      float* w_out, int64_t N, int64_t K, q4_stream_t stream) {
+    q4_status st = check_K(K);
+    if (st != Q4_OK) return st;
+    if (N < 0 || N > Q4_MAX_MN) return Q4_ERR_SHAPE;
+    if (N == 0) return Q4_OK;
+    if (!codes || !scales || !codebook4 || !w_out) return Q4_ERR_NULL;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(codebook4) || !aligned16(w_out))
+        return Q4_ERR_ALIGN;
+    DeviceInfo dev;
+    if ((st = gate(&dev)) != Q4_OK) return st;
+    return after_launch(launch_dequant2(codes, scales, codebook4, w_out, N, K, stream, dev));
+}
+
+q4_status q4_gemv2(const uint8_t* codes, const uint16_t* scales, const uint16_t* codebook4,
+                   const uint16_t* x, float* y, int64_t N, int64_t K, q4_stream_t stream) {
+    if (K > Q4_GEMV2_MAX_K) return Q4_ERR_SHAPE;
+    bool empty;
+    q4_status st = check_matmul(codes, scales, codebook4, x, y, 1, N, K, &empty);
+    if (st != Q4_OK || empty) return st;
+    DeviceInfo dev;
+    if ((st = gate(&dev)) != Q4_OK) return st;
+    cudaError_t e = launch_gemv2(codes, scales, codebook4, x, y, N, K, stream, dev);
+    if (e == cudaErrorNotSupported) {
+        (void)cudaGetLastError();
+        return Q4_ERR_SHAPE;
+    }
+    return after_launch(e);
+}
+
 q4_status q4_timeout_flags(uint32_t* flags) {
     if (!flags) return Q4_ERR_NULL;
     *flags = 0;

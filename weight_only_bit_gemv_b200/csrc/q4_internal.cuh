@@ -68,6 +68,18 @@ cudaError_t launch_prefill_noalloc(const uint8_t* codes, const uint16_t* scales,
                                    const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
                                    cudaStream_t s, const DeviceInfo& dev);
 
+// The two-bit variant (q2_codebook.cu): codes [N][K/4], a 4-entry codebook.
+cudaError_t launch_pack2(const float* w, const uint16_t* cb, uint8_t* codes, uint16_t* scales,
+                         int64_t N, int64_t K, cudaStream_t s, const DeviceInfo& dev);
+cudaError_t launch_dequant2(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                            float* w, int64_t N, int64_t K, cudaStream_t s, const DeviceInfo& dev);
+// One token; zeroes y on the stream, then adds into it.  Returns
+// cudaErrorNotSupported when the staged x (136 bytes per group) does not fit
+// the device's shared memory.
+cudaError_t launch_gemv2(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                         const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
+                         const DeviceInfo& dev);
+
 // Copy out and clear the timeout bits that a kernel family's bounded waits
 // set (synchronous; see q4_timeout_flags).
 cudaError_t take_gemv_m1_error(unsigned int* out);
