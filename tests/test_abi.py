@@ -139,3 +139,20 @@ def test_binding_marshalling_checks():
                    torch.zeros(1, 64, dtype=torch.bfloat16))
     with pytest.raises(TypeError):
         q4.q4_pack(torch.zeros(4, 64, dtype=torch.float64), torch.zeros(16, dtype=torch.float16))
+
+
+def test_two_bit_binding_marshalling_checks():
+    import torch
+    codes = torch.zeros(4, 16, dtype=torch.uint8)              # N = 4, K = 64
+    scales = torch.zeros(4, 1, dtype=torch.float16)
+    cb4 = torch.zeros(4, dtype=torch.float16)
+    with pytest.raises(ValueError):                            # x of the wrong K
+        q4.q4_gemv2(codes, scales, cb4, torch.zeros(1, 128, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):                            # M != 1
+        q4.q4_gemv2(codes, scales, cb4, torch.zeros(2, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):                            # host tensors
+        q4.q4_gemv2(codes, scales, cb4, torch.zeros(1, 64, dtype=torch.bfloat16))
+    with pytest.raises(TypeError):
+        q4.q4_pack2(torch.zeros(4, 64, dtype=torch.float64), cb4)
+    with pytest.raises(ValueError):                            # codes not 2-D
+        q4.q4_dequant2(torch.zeros(64, dtype=torch.uint8), scales, cb4)
