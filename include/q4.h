@@ -1,6 +1,6 @@
 /*
  * q4.h -- C ABI of the weight-only 4-bit codebook linear layer for NVIDIA
- * B200 (sm_100a).
+ * B200 (sm_100a), with a two-bit variant (q4_pack2, q4_dequant2, q4_gemv2).
  *
  * The operation.  A linear layer y = x * W^T whose weight matrix W [N][K]
  * (N outputs, K inputs) is stored as 4-bit codes into a 16-entry binary16
