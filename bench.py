@@ -176,6 +176,15 @@ def aggregate(units_per_rank, ms_per_step, world):
 # the layer on the GPU
 # ---------------------------------------------------------------------------
 
+def pcts(ms_list):
+    """[p10, median, p90] of a list of durations in ms, in µs."""
+    med = statistics.median(ms_list)
+    if len(ms_list) < 2:
+        return [round(med * 1e3, 3)] * 3
+    q = statistics.quantiles(ms_list, n=10, method="inclusive")
+    return [round(q[0] * 1e3, 3), round(med * 1e3, 3), round(q[8] * 1e3, 3)]
+
+
 def build_layer(dev, cb):
     import torch
     import weight_only_bit_gemv_b200 as q4
@@ -375,6 +384,12 @@ def run_ours(args, world, rank, local):
     embed = None if args.no_smallm else bench_embed_rows(dev, cb, stream, hbm_peak)
     ring = None if args.no_smallm else bench_ring(dev, cb, stream, lins)
     two_bit = None if args.no_smallm else bench_gemv2(dev, stream, hbm_peak)
+    bf16_base = None
+    if not args.no_gemm:
+        try:
+            bf16_base = bench_bf16_baseline(dev, cb, stream, lins, hbm_peak, tc_peak, ms_step, gemm)
+        except Exception as exc:  # a baseline must not cost the bench line
+            bf16_base = {"error": f"{type(exc).__name__}: {exc}"[:300]}
 
     # ---- CPU baseline: the oracle on the host --------------------------------
     cpu = None
@@ -404,6 +419,7 @@ def run_ours(args, world, rank, local):
             "launch": "CUDA graphs of the step's four launches",
             "hbm_frac_of_" + peak_src: round(value / world / hbm_peak, 4),
             "per_linear_us": {L["lin"].name: round(per_ms[j] * 1e3, 3) for j, L in enumerate(lins)},
+            "per_linear_us_p10_p50_p90": {L["lin"].name: pcts(per[j]) for j, L in enumerate(lins)},
             "decode_tok_s_equiv_32_layers": round(1e3 / (ms_step * 32), 1),
         },
         "roofline": {
@@ -445,6 +461,8 @@ def run_ours(args, world, rank, local):
         line["copy_ring"] = ring
     if two_bit is not None:
         line["two_bit_gemv_llama2_70b"] = two_bit
+    if bf16_base is not None:
+        line["torch_bf16_baseline"] = bf16_base
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if rank == 0:
@@ -666,6 +684,86 @@ def bench_embed_rows(dev, cb, stream, hbm_peak, n_ids=4096, reps=20):
             "us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
             "hbm_frac_of_measured": round(gbs / hbm_peak, 4),
             "timing": "CUDA graph of 4 calls on different ids, replayed 20 times"}
+
+
+def _graph_time_ms(fn, stream, per=4, reps=10):
+    """Device time of one ``fn()`` call: a CUDA graph of ``per`` calls,
+    replayed ``reps`` times after an eager warm-up."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            fn()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(per):
+            fn()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g.replay()
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+    e1.synchronize()
+    del g
+    return e0.elapsed_time(e1) / (reps * per)
+
+
+def bench_bf16_baseline(dev, cb, stream, lins, hbm_peak, tc_peak, ours_ms_step, gemm):
+    """The same shapes in plain torch: y = x @ W_bf16^T through cuBLAS, with
+    W_bf16 = bf16(dequantized W), i.e. 2 B per weight.  Decode: the
+    Llama-2-7B layer at M = 1 against the q4_gemv step; prefill: the
+    Llama-2-70B layer at M = 256 against q4_gemm."""
+    import torch
+    import weight_only_bit_gemv_b200 as q4
+    # decode, M = 1
+    ws = [q4.q4_dequant(L["copies"][0][0], L["copies"][0][1], cb).to(torch.bfloat16) for L in lins]
+    ys = [torch.empty((1, L["lin"].N), dtype=torch.bfloat16, device=dev) for L in lins]
+
+    def step():
+        for L, w, y in zip(lins, ws, ys):
+            torch.matmul(L["x"], w.t(), out=y)
+
+    ms = _graph_time_ms(step, stream, per=4, reps=20)
+    nbytes = sum(2 * L["lin"].N * L["lin"].K + 2 * L["lin"].K + 2 * L["lin"].N for L in lins)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out = {"decode_llama2_7b_layer_m1": {
+        "us_per_step": round(ms * 1e3, 2), "gbs_at_2B_per_weight": round(gbs, 1),
+        "hbm_frac_of_measured": round(gbs / hbm_peak, 4),
+        "q4_gemv_speedup": round(ms / ours_ms_step, 3)}}
+    del ws, ys
+    torch.cuda.empty_cache()
+    # prefill, M = 256
+    M = 256
+    wl = synth.WORKLOADS["llama2_70b_prefill"]
+    tot_ms, tot_flop, per_lin = 0.0, 0.0, {}
+    for lin in wl.linears:
+        seed = synth.seed_for(wl.index, 0, lin.name)
+        w = synth.weights_device(seed, lin.N, lin.K, wl.w_std, dev)
+        codes, scales = q4.q4_pack(w, cb)
+        del w
+        wb = q4.q4_dequant(codes, scales, cb).to(torch.bfloat16)
+        del codes, scales
+        x = synth.activations_device(synth.x_seed(seed) + M, M, lin.K, dev)
+        y = torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev)
+        lms = _graph_time_ms(lambda: torch.matmul(x, wb.t(), out=y), stream, per=4, reps=5)
+        flop = 2.0 * M * lin.N * lin.K
+        per_lin[lin.name] = {"us": round(lms * 1e3, 2), "tflops": round(flop / (lms * 1e-3) / 1e12, 2)}
+        tot_ms += lms
+        tot_flop += flop
+        del wb, x, y
+        torch.cuda.empty_cache()
+    tf = tot_flop / (tot_ms * 1e-3) / 1e12
+    pre = {"tflops": round(tf, 2), "frac_of_bf16_peak": round(tf / tc_peak, 4),
+           "us_per_layer": round(tot_ms * 1e3, 2), "per_linear": per_lin}
+    if gemm is not None:
+        pre["q4_gemm_speedup"] = round(gemm["tflops"] / tf, 3)
+    out["prefill_llama2_70b_layer_m256"] = pre
+    out["timing"] = ("CUDA graphs of 4 calls (decode: 4 steps of the 4 linears), replayed 20 (decode) "
+                     "or 5 (prefill) times; bf16 output; W_bf16 = bf16(q4_dequant(codes, scales))")
+    return out
 
 
 def bench_gemv2(dev, stream, hbm_peak, reps=20):

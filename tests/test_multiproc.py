@@ -78,3 +78,12 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.aggregate(10.0, 2.0, 1) == pytest.approx(5000.0)
+
+
+def test_percentile_helper():
+    import bench
+    ms = [i / 1000.0 for i in range(1, 102)]        # 1..101 µs
+    p10, p50, p90 = bench.pcts(ms)
+    assert p50 == pytest.approx(51.0)
+    assert p10 == pytest.approx(11.0) and p90 == pytest.approx(91.0)
+    assert bench.pcts([0.002]) == [2.0, 2.0, 2.0]
