@@ -57,12 +57,13 @@ cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const u
 cudaError_t launch_gemm_small(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                               const uint16_t* x, float* y, int M, int64_t N, int64_t K,
                               cudaStream_t s, const DeviceInfo& dev);
-// M > 16: tcgen05 tensor-core GEMM with TMEM accumulators.
+// M > 24 (and M = 17..24 when launch_gemm_small declines the shape):
+// tcgen05 tensor-core GEMM with TMEM accumulators.
 cudaError_t launch_prefill(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
                            cudaStream_t s, const DeviceInfo& dev);
 
-// M > 16 with the x scratch in a fixed device array (q4_gemm_noalloc); the
+// launch_prefill with the x scratch in a fixed device array (q4_gemm_noalloc); the
 // caller has checked 2 * M * K <= Q4_NOALLOC_SCRATCH_BYTES.
 cudaError_t launch_prefill_noalloc(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                                    const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
