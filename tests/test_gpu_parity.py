@@ -180,6 +180,22 @@ def test_gemv2_integer_codebook_exact():
     assert np.array_equal(y.cpu().numpy(), y_ref)
 
 
+def test_gemv2_output_bounds_and_stream():
+    """q4_gemv2 zeroes and adds into y only: canaries on both sides stay, and
+    a side stream orders its memset and kernel."""
+    N, K = 77, 320
+    codes, scales = synth.tiny_codes2_scales(13, N, K)
+    x = synth.activations(14, 1, K)
+    buf = torch.full((N + 32,), 12345.0, dtype=torch.float32, device="cuda")
+    y = buf[16:16 + N].view(1, N)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        q4.q4_gemv2(dev_u8(codes), dev_u16(scales), dev_u16(CB4), dev_u16(x), y)
+    s.synchronize()
+    assert torch.all(buf[:16] == 12345.0) and torch.all(buf[16 + N:] == 12345.0)
+    assert_close2(y.cpu().numpy(), codes, scales, x, label="gemv2 stream")
+
+
 @pytest.mark.parametrize("linear", ["qkv", "o", "gate_up", "down"])
 def test_gemv2_llama2_70b_layer(linear):
     """The Llama-2-70B decoder layer's linears in 2 bits at M = 1: 1024 sampled
