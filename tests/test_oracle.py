@@ -475,6 +475,37 @@ def pin_two_bit_pack_ties(o):
     assert got == [3, 0, 1, 2]
 
 
+def pin_two_bit_codebook_permutation(o):
+    """Permuting the codebook and inverse-permuting the codes leaves W, and
+    so y, unchanged (the codebook is looked up, never assumed sorted)."""
+    rng = np.random.default_rng(25)
+    N, K = 5, 2 * GROUP
+    codes = rng.integers(0, 256, size=(N, K // 4), dtype=np.uint8)
+    scales = synth.f32_to_f16_bits(rng.uniform(0.005, 0.05, size=(N, K // GROUP)).astype(np.float32))
+    perm = np.array([2, 0, 3, 1])                       # new entry j = old entry perm[j]
+    inv = np.argsort(perm)                              # old index c -> new index inv[c]
+    cb_p = CB4[perm]
+    codes_p = np.zeros_like(codes)
+    for i in range(4):
+        codes_p |= (inv[(codes >> (2 * i)) & 3].astype(np.uint8) << (2 * i))
+    assert np.array_equal(o.dequant2(codes_p, scales, cb_p), o.dequant2(codes, scales, CB4))
+    x = synth.f32_to_bf16_bits(rng.standard_normal((1, K)).astype(np.float32))
+    assert np.array_equal(o.matmul2(codes_p, scales, cb_p, x)[0], o.matmul2(codes, scales, CB4, x)[0])
+
+
+def pin_two_bit_matmul_one_hot(o):
+    """x = e_k picks column k of W exactly."""
+    rng = np.random.default_rng(26)
+    N, K = 9, 3 * GROUP
+    codes = rng.integers(0, 256, size=(N, K // 4), dtype=np.uint8)
+    scales = synth.f32_to_f16_bits(rng.uniform(0.005, 0.05, size=(N, K // GROUP)).astype(np.float32))
+    W = _decode2_numpy(codes, scales, CB4)
+    for k in (0, 1, 63, 64, K - 1):
+        x = np.zeros((1, K), np.uint16)
+        x[0, k] = 0x3F80                                  # bf16 1.0
+        assert np.array_equal(o.matmul2(codes, scales, CB4, x)[0][0], W[:, k])
+
+
 def pin_two_bit_matmul_brute_force(o):
     rng = np.random.default_rng(24)
     N, K, M = 11, 2 * GROUP, 3
