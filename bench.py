@@ -721,6 +721,7 @@ def bench_bf16_baseline(dev, cb, stream, lins, hbm_peak, tc_peak, ours_ms_step, 
     # decode, M = 1
     ws = [q4.q4_dequant(L["copies"][0][0], L["copies"][0][1], cb).to(torch.bfloat16) for L in lins]
     ys = [torch.empty((1, L["lin"].N), dtype=torch.bfloat16, device=dev) for L in lins]
+    torch.cuda.synchronize()  # the weights were made on the default stream
 
     def step():
         for L, w, y in zip(lins, ws, ys):
@@ -748,6 +749,7 @@ def bench_bf16_baseline(dev, cb, stream, lins, hbm_peak, tc_peak, ours_ms_step, 
         del codes, scales
         x = synth.activations_device(synth.x_seed(seed) + M, M, lin.K, dev)
         y = torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
         lms = _graph_time_ms(lambda: torch.matmul(x, wb.t(), out=y), stream, per=4, reps=5)
         flop = 2.0 * M * lin.N * lin.K
         per_lin[lin.name] = {"us": round(lms * 1e3, 2), "tflops": round(flop / (lms * 1e-3) / 1e12, 2)}
@@ -782,6 +784,7 @@ def bench_gemv2(dev, stream, hbm_peak, reps=20):
         x = synth.activations_device(synth.x_seed(synth.seed_for(5, 0, lin.name)), 1, lin.K, dev)
         y = torch.empty((1, lin.N), dtype=torch.float32, device=dev)
         lins.append((lin, codes, scales, x, y))
+    torch.cuda.synchronize()  # inputs drawn on the default stream
     with torch.cuda.stream(stream):
         for lin, c, sc, x, y in lins:
             q4.q4_gemv2(c, sc, cb4, x, y)
