@@ -156,3 +156,12 @@ def test_two_bit_binding_marshalling_checks():
         q4.q4_pack2(torch.zeros(4, 64, dtype=torch.float64), cb4)
     with pytest.raises(ValueError):                            # codes not 2-D
         q4.q4_dequant2(torch.zeros(64, dtype=torch.uint8), scales, cb4)
+
+
+def test_binding_has_every_header_name():
+    """The binding exposes each entry point of include/q4.h under its C name."""
+    missing = [n for n in q4.header_functions() if not callable(getattr(q4, n, None))]
+    assert not missing, missing
+    assert q4.q4_abi_version() == q4.abi_version()
+    assert q4.q4_status_string(0) == q4.status_string(0)
+    assert isinstance(q4.q4_last_cuda_error(), int)

@@ -355,3 +355,34 @@ def timeout_flags() -> int:
 
 def abi_version() -> int:
     return load().q4_abi_version()
+
+
+# ---- the C names, one Python function per entry point of include/q4.h ------
+
+def q4_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def q4_last_cuda_error() -> int:
+    """The CUDA error code behind the calling thread's last Q4_ERR_CUDA."""
+    return int(load().q4_last_cuda_error())
+
+
+def q4_abi_version() -> int:
+    return abi_version()
+
+
+def q4_timeout_flags() -> int:
+    return timeout_flags()
+
+
+def q4_ring_create(slot_bytes: int) -> Ring:
+    return Ring(slot_bytes)
+
+
+def q4_ring_gemm(ring: Ring, codes_host, scales_host, codebook, x, y=None, stream=None):
+    return ring.gemm(codes_host, scales_host, codebook, x, y, stream)
+
+
+def q4_ring_destroy(ring: Ring) -> None:
+    ring.close()
