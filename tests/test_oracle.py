@@ -324,7 +324,7 @@ def pin_matmul_integer_exact(o):
     x = synth.f32_to_bf16_bits(xi.astype(np.float32))
     y, _ = o.matmul(pack_codes(c), scales, cb, x)
     Wi = (c.astype(np.int64) - 8) * np.repeat(2 ** e, GROUP, axis=1)
-    assert np.all(np.isfinite(y)) and np.all(y == np.round(y))
+    assert np.all(np.isfinite(y)) and np.all(y == np.round(y)) and np.all(np.abs(y) < 2.0 ** 62)
     assert np.array_equal(y.astype(np.int64), xi @ Wi.T)
 
 
