@@ -22,6 +22,8 @@
  *  - "Trapetum" overview, "What it does": the fused kernel reads the weights
  *    straight out of the codebook.  "Trapetum" landing page: the matrix is
  *    decoded inside the matmul and never materialized.
+ *  - "Trapetum" overview, "In one sentence" and "Frontier models on your own
+ *    hardware": a 70B model in 2 bits (the two-bit variant below).
  *  - NF4 (NormalFloat, QLoRA): sixteen quantiles of the standard normal,
  *    asymmetric (8 positive, 7 negative, an exact zero), scaled to [-1, 1].
  *
