@@ -404,6 +404,15 @@ def test_small_m_verify(linear, M):
     assert_close(y, codes, scales, NF4, x, rows=rows, label=f"{linear} M={M}")
 
 
+@pytest.mark.parametrize("linear", ["qkv", "o", "gate_up", "down"])
+def test_small_m_verify_full_m16(linear):
+    """The widest verify batch in full: M = 16, every output of each
+    Llama-3.1-8B layer linear."""
+    w, codes, scales, seed = packed_linear("llama31_8b_step", linear)
+    x = synth.activations(synth.x_seed(seed) + 16, 16, codes.shape[1] * 2)
+    assert_close(run_matmul(codes, scales, NF4, x), codes, scales, NF4, x, label=f"{linear} M=16 full")
+
+
 @pytest.mark.parametrize("M", [32, 128, 256, 512])
 @pytest.mark.parametrize("linear", ["qkv", "o", "gate_up", "down"])
 def test_llama2_70b_prefill(linear, M):
