@@ -11,9 +11,9 @@
  * This is the layout the "deep-fold" page describes in its "Method" section
  * (each group of 64 weights stores four-bit NF4 codes and one FP16 scale;
  * the packed payload is about 3.76x smaller than BF16).  The matmul entry
- * points rebuild W inside the kernel while they multiply, reading the codes
- * "straight out of the codebook" ("Trapetum" overview, "What it does"), and
- * never write a dense W to memory ("Trapetum" landing page, opening
+ * points rebuild W inside the kernel while they multiply, decoding each
+ * weight from the codebook as it is used ("Trapetum" overview, "What it
+ * does"), and never write a dense W to memory ("Trapetum" landing page, opening
  * paragraph; "deep-fold", "Method").  Decode (one token) is a GEMV and
  * prompt processing a tensor-core GEMM ("deep-fold", "Method" table).
  *
@@ -300,13 +300,72 @@ q4_status q4_gemv2(const uint8_t* codes, const uint16_t* scales,
                    int64_t N, int64_t K, q4_stream_t stream);
 
 /*
+ * Decode steps as one CUDA graph.
+ * Source: "deep-fold", "Method" table (the decode runs a full greedy step as
+ * one CUDA graph); "Trapetum" landing page (the 7B decode rate it reports
+ * with CUDA graphs).  A decode step launches the same linears on the same
+ * buffers token after token; recording those launches once and replaying
+ * them removes the host's launch cost from every token.
+ *
+ * q4_linear -- one linear of a step: y = x W^T with the arguments of q4_gemm
+ * (M = 1 runs q4_gemv's kernel).  The pointers are baked into the step: to
+ * run the next token, write new values into the same x buffers and launch
+ * the step again.
+ *
+ * q4_step_create -- validate every linear as q4_gemm does (the first failure
+ * is returned, and nothing is recorded), then record their launches, in list
+ * order, on a private stream of the current device into a CUDA graph and
+ * instantiate it.  Nothing runs.  Consecutive launches keep programmatic
+ * dependent launch, so a kernel's start overlaps the end of the one before.
+ * Linears with M == 0 or N == 0 are skipped.  Creates a stream and a graph
+ * (host-side objects and the driver's own graph resources); no device memory
+ * is allocated for the linears' data.  Returns Q4_ERR_NULL for a NULL list
+ * or step, Q4_ERR_SHAPE for n < 1, the linears' validation errors,
+ * Q4_ERR_ARCH, Q4_ERR_CUDA.
+ *
+ * q4_step_launch -- replay the recorded launches on `stream` (asynchronous;
+ * the step's device must be current).  Replays on different streams that
+ * overlap race on the linears' y buffers.
+ *
+ * q4_step_destroy -- free the graph and the stream (waits for nothing: let
+ * the step's launches finish first).
+ */
+typedef struct {
+    const uint8_t* codes;
+    const uint16_t* scales;
+    const uint16_t* codebook;
+    const uint16_t* x;
+    float* y;
+    int64_t M, N, K;
+} q4_linear;
+typedef struct q4_step q4_step;
+q4_status q4_step_create(const q4_linear* linears, int64_t n, q4_step** step);
+q4_status q4_step_launch(q4_step* step, q4_stream_t stream);
+q4_status q4_step_destroy(q4_step* step);
+
+/*
+ * q4_wait_selftest -- exercise the bounded wait the kernels use, with
+ * nothing in flight: one thread block initializes an mbarrier that expects
+ * one arrival, arrives on it only if `arrive` is nonzero, and waits on it for
+ * at most limit_us microseconds (1..1000000) of the GPU's global timer.  A
+ * wait that runs out sets bit 7 of q4_timeout_flags, exactly as a kernel's
+ * wait that runs out sets its own bit, and the block returns.  The call
+ * synchronizes the current device and stores in *waited_us how long the wait
+ * took.  Not an operation of the method: a check of the failure detection.
+ * Returns Q4_ERR_NULL for a NULL waited_us, Q4_ERR_SHAPE for a limit outside
+ * 1..1000000, Q4_ERR_ARCH, Q4_ERR_CUDA.
+ */
+q4_status q4_wait_selftest(uint32_t limit_us, int arrive, uint32_t* waited_us);
+
+/*
  * q4_timeout_flags -- every wait inside the bulk-copy and tensor-core
  * kernels is bounded (about two seconds); a wait that runs out sets a bit in
  * a device word, the kernel drains what it has in flight, frees its tensor
  * memory and exits, leaving its output incomplete.  This call synchronizes the
  * current device, stores the bits set since the last call in *flags and
- * clears them: bits 0-11 the M = 1 GEMV (bit 8: its shared-memory layout did
- * not match the device; bits 9-11: producer, drain and consumer waits), bits
+ * clears them: bits 0-11 the M = 1 GEMV (bit 7: q4_wait_selftest's wait ran
+ * out; bit 8: its shared-memory layout did not match the device; bits 9-11:
+ * producer, drain and consumer waits), bits
  * 12-15 the M = 2..24 kernel (the same four conditions), bits 16-31 the
  * tensor-core GEMM (M > 24); 0 = none.  Not an operation of the method; a
  * health check.

@@ -19,8 +19,8 @@
  *    tensor-core GEMM.
  *  - Same page, introduction and Figure 1: embeddings (PackedEmbed) decode
  *    only the requested rows, on a path of their own.
- *  - "Trapetum" overview, "What it does": the fused kernel reads the weights
- *    straight out of the codebook.  "Trapetum" landing page: the matrix is
+ *  - "Trapetum" overview, "What it does": the fused kernel decodes each
+ *    weight from the codebook as it multiplies.  "Trapetum" landing page: the matrix is
  *    decoded inside the matmul and never materialized.
  *  - "Trapetum" overview, "In one sentence" and "Frontier models on your own
  *    hardware": a 70B model in 2 bits (the two-bit variant below).

@@ -48,3 +48,24 @@ def within_tolerance(y_test, y_ref, absacc, rel=1e-4, abs_=1e-6):
     ok = bool(np.all(err <= bound)) and bool(np.all(np.isfinite(y_test)))
     worst = float(np.max(err / bound)) if err.size else 0.0
     return ok, worst
+
+
+def oracle_matmul_parallel(codes, scales, cb, x, rows=None, workers=None):
+    """oracle.matmul on the given rows of W (all rows if None), split into
+    chunks run on host threads.  The oracle is a C library called through
+    ctypes, which releases the GIL for the call, so the chunks run on as many
+    cores as there are workers; each chunk is the oracle's own serial loop.
+    Returns (y [M, n_rows] fp32, sum|W x| [M, n_rows] fp64)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle
+
+    N = codes.shape[0]
+    rows = np.arange(N, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    workers = workers or max(1, min(32, os.cpu_count() or 1))
+    chunks = [c for c in np.array_split(rows, workers) if c.size]
+    with ThreadPoolExecutor(max_workers=len(chunks)) as ex:
+        parts = list(ex.map(lambda c: oracle.matmul(codes, scales, cb, x, rows=c), chunks))
+    return (np.concatenate([p[0] for p in parts], axis=1),
+            np.concatenate([p[1] for p in parts], axis=1))

@@ -165,3 +165,29 @@ def test_binding_has_every_header_name():
     assert q4.q4_abi_version() == q4.abi_version()
     assert q4.q4_status_string(0) == q4.status_string(0)
     assert isinstance(q4.q4_last_cuda_error(), int)
+
+
+def test_step_rejects(lib):
+    """q4_step_create validates its list (and every linear as q4_gemm does)
+    before it records anything."""
+    h = ctypes.c_void_p()
+    L = q4.Q4Linear
+    good = L(A, A, A, A, A, 1, 64, 256)
+    assert lib.q4_step_create((L * 1)(good), 1, None) == NULL
+    assert lib.q4_step_create(None, 1, ctypes.byref(h)) == NULL
+    assert lib.q4_step_create((L * 1)(good), 0, ctypes.byref(h)) == SHAPE
+    assert lib.q4_step_create((L * 2)(good, L(A, A, A, A, A, 1, 64, 100)), 2,
+                              ctypes.byref(h)) == SHAPE             # second linear: K % 64
+    assert lib.q4_step_create((L * 2)(good, L(A, A, None, A, A, 4, 64, 64)), 2,
+                              ctypes.byref(h)) == NULL
+    assert lib.q4_step_create((L * 1)(L(A, A, A, MIS, A, 2, 64, 64)), 1, ctypes.byref(h)) == ALIGN
+    assert h.value is None
+    assert lib.q4_step_launch(None, None) == NULL
+    assert lib.q4_step_destroy(None) == NULL
+
+
+def test_wait_selftest_rejects(lib):
+    out = ctypes.c_uint32(7)
+    assert lib.q4_wait_selftest(1000, 0, None) == NULL
+    assert lib.q4_wait_selftest(0, 0, ctypes.byref(out)) == SHAPE
+    assert lib.q4_wait_selftest(1000001, 1, ctypes.byref(out)) == SHAPE

@@ -14,10 +14,9 @@ import numpy as np
 import pytest
 import torch
 
-import oracle
 import synth
 import weight_only_bit_gemv_b200 as q4
-from helpers import GROUP
+from helpers import GROUP, oracle_matmul_parallel, within_tolerance
 
 pytestmark = pytest.mark.gpu
 
@@ -55,20 +54,40 @@ def _case(seed, M, N, K):
     return codes, scales, x
 
 
-def test_matches_q4_gemm_on_two_calls_in_a_row():
+def _compare(seed, M, N, K, cb):
+    """q4_gemm_noalloc against the oracle's y and against q4_gemm's y, both
+    within the parity tolerance."""
+    codes, scales, x = _case(seed, M, N, K)
+    c, s, xd = torch.from_numpy(codes).cuda(), _dev16(scales), _dev16(x)
+    y_gemm = torch.full((M, N), float("nan"), device="cuda")
+    y_new = torch.full((M, N), float("nan"), device="cuda")
+    assert _call("q4_gemm", c, s, cb, xd, y_gemm) == 0
+    assert _call("q4_gemm_noalloc", c, s, cb, xd, y_new) == 0
+    y_ref, absacc = oracle_matmul_parallel(codes, scales, NF4, x)
+    new, old = y_new.cpu().numpy(), y_gemm.cpu().numpy()
+    ok, worst = within_tolerance(new, y_ref, absacc)
+    assert ok, f"M={M} N={N} K={K}: against the oracle, worst err/bound = {worst:.3g}"
+    ok, worst = within_tolerance(new, old, absacc)
+    assert ok, f"M={M} N={N} K={K}: against q4_gemm, worst err/bound = {worst:.3g}"
+
+
+def test_matches_oracle_on_two_calls_in_a_row():
     cb = _dev16(NF4)
     # the second call is smaller and has other data: stale scratch must not matter
     for seed, (M, N, K) in ((21, (96, 300, 4096)), (22, (40, 130, 1088))):
-        codes, scales, x = _case(seed, M, N, K)
-        c, s, xd = torch.from_numpy(codes).cuda(), _dev16(scales), _dev16(x)
-        y_ref = torch.full((M, N), float("nan"), device="cuda")
-        y_new = torch.full((M, N), float("nan"), device="cuda")
-        assert _call("q4_gemm", c, s, cb, xd, y_ref) == 0
-        assert _call("q4_gemm_noalloc", c, s, cb, xd, y_new) == 0
-        _, absacc = oracle.matmul(codes, scales, NF4, x)
-        a, b = y_new.cpu().numpy().astype(np.float64), y_ref.cpu().numpy().astype(np.float64)
-        assert np.all(np.isfinite(a))
-        assert np.all(np.abs(a - b) <= 1e-4 * absacc + 1e-6), f"M={M} N={N} K={K}"
+        _compare(seed, M, N, K, cb)
+    assert q4.timeout_flags() == 0
+
+
+def test_verify_sizes_and_exact_fit():
+    """M = 20 (the M <= 24 kernel, which needs no scratch) and the largest
+    input that fits: 2 * M * K equal to the array's size (M = 512, K = 8192),
+    which would expose an access one past its end."""
+    cb = _dev16(NF4)
+    _compare(24, 20, 257, 4160, cb)
+    assert 2 * 512 * 8192 == SCRATCH
+    _compare(25, 512, 130, 8192, cb)
+    assert q4.timeout_flags() == 0
 
 
 def test_small_m_and_size_limit():
@@ -79,9 +98,9 @@ def test_small_m_and_size_limit():
     y_new = torch.empty((8, 64), device="cuda")
     assert _call("q4_gemm", c, s, cb, xd, y_ref) == 0
     assert _call("q4_gemm_noalloc", c, s, cb, xd, y_new) == 0
-    _, absacc = oracle.matmul(codes, scales, NF4, x)
-    a, b = y_new.cpu().numpy().astype(np.float64), y_ref.cpu().numpy().astype(np.float64)
-    assert np.all(np.abs(a - b) <= 1e-4 * absacc + 1e-6)
+    y_or, absacc = oracle_matmul_parallel(codes, scales, NF4, x)
+    assert within_tolerance(y_new.cpu().numpy(), y_or, absacc)[0]
+    assert within_tolerance(y_new.cpu().numpy(), y_ref.cpu().numpy(), absacc)[0]
     # one token past the limit is refused before anything runs
     K = 4096
     M = SCRATCH // (2 * K) + 1

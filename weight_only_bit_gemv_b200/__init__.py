@@ -40,6 +40,13 @@ class Q4Error(RuntimeError):
 _lib = None
 
 
+class Q4Linear(ctypes.Structure):
+    """struct q4_linear of q4.h: one linear of a recorded step."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("codebook", ctypes.c_void_p), ("x", ctypes.c_void_p), ("y", ctypes.c_void_p),
+                ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
 def library_path() -> str:
     return _build.LIBRARY
 
@@ -82,6 +89,14 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.q4_ring_gemm.restype = ctypes.c_int
     lib.q4_ring_destroy.argtypes = [P]
     lib.q4_ring_destroy.restype = ctypes.c_int
+    lib.q4_step_create.argtypes = [ctypes.POINTER(Q4Linear), I64, ctypes.POINTER(ctypes.c_void_p)]
+    lib.q4_step_create.restype = ctypes.c_int
+    lib.q4_step_launch.argtypes = [P, S]
+    lib.q4_step_launch.restype = ctypes.c_int
+    lib.q4_step_destroy.argtypes = [P]
+    lib.q4_step_destroy.restype = ctypes.c_int
+    lib.q4_wait_selftest.argtypes = [ctypes.c_uint32, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32)]
+    lib.q4_wait_selftest.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -346,6 +361,63 @@ class Ring:
             pass
 
 
+class Step:
+    """A decode step recorded once as a CUDA graph (q4_step_create) and
+    replayed per token (``launch``).  ``linears`` is a sequence of
+    (codes, scales, codebook, x, y) device tensors with the q4_gemm
+    conventions; the graph keeps their addresses, so the caller keeps the
+    tensors alive and writes each token's activations into the same x."""
+
+    def __init__(self, linears):
+        self._keep = []
+        arr = (Q4Linear * len(linears))()
+        for i, (codes, scales, codebook, x, y) in enumerate(linears):
+            N, K = _packed_dims(codes)
+            if x.dim() != 2 or x.shape[1] != K:
+                raise ValueError(f"linear {i}: x must be [M, {K}]")
+            M = x.shape[0]
+            _need(codes, "codes", (torch.uint8,))
+            _need(scales, "scales", _H16, (N, K // GROUP))
+            _need(codebook, "codebook", _H16, (16,))
+            _need(x, "x", _BF16)
+            _need(y, "y", (torch.float32,), (M, N))
+            arr[i] = Q4Linear(codes.data_ptr(), scales.data_ptr(), codebook.data_ptr(),
+                              x.data_ptr(), y.data_ptr(), M, N, K)
+            self._keep.append((codes, scales, codebook, x, y))
+        self._device = self._keep[0][0].device if self._keep else None
+        self._h = ctypes.c_void_p()
+        _check(load().q4_step_create(arr, len(linears), ctypes.byref(self._h)), "q4_step_create")
+
+    def launch(self, stream=None) -> None:
+        if self._h.value is None:
+            raise RuntimeError("step is closed")
+        if stream is None:
+            stream = torch.cuda.current_stream(self._device)
+        s = int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+        _check(load().q4_step_launch(self._h, s), "q4_step_launch")
+
+    def close(self) -> None:
+        if self._h.value is not None:
+            _check(load().q4_step_destroy(self._h), "q4_step_destroy")
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def wait_selftest(limit_us: int, arrive: bool) -> int:
+    """Run the bounded-wait self-test kernel (synchronizes the device); returns
+    the microseconds the wait took.  Without ``arrive`` the wait runs out and
+    sets bit 7 of timeout_flags()."""
+    out = ctypes.c_uint32(0)
+    _check(load().q4_wait_selftest(int(limit_us), 1 if arrive else 0, ctypes.byref(out)),
+           "q4_wait_selftest")
+    return int(out.value)
+
+
 def timeout_flags() -> int:
     """Synchronize the current device; return and clear the kernels' bounded-wait timeout bits."""
     out = ctypes.c_uint32(0)
@@ -386,3 +458,19 @@ def q4_ring_gemm(ring: Ring, codes_host, scales_host, codebook, x, y=None, strea
 
 def q4_ring_destroy(ring: Ring) -> None:
     ring.close()
+
+
+def q4_step_create(linears) -> Step:
+    return Step(linears)
+
+
+def q4_step_launch(step: Step, stream=None) -> None:
+    step.launch(stream)
+
+
+def q4_step_destroy(step: Step) -> None:
+    step.close()
+
+
+def q4_wait_selftest(limit_us: int, arrive: bool) -> int:
+    return wait_selftest(limit_us, arrive)

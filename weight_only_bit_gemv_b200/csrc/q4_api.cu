@@ -146,6 +146,12 @@ struct q4_ring {
     int next = 0;
 };
 
+// A recorded decode step (see q4_step_create in q4.h).
+struct q4_step {
+    int device = 0;
+    cudaStream_t capture = nullptr;
+    cudaGraphExec_t exec = nullptr;
+};
 
 extern "C" {
 
@@ -328,6 +334,80 @@ q4_status q4_ring_gemm(q4_ring* ring, const uint8_t* host_codes, const uint16_t*
     if (e != cudaSuccess) return cuda_fail(e);
     ring->next = s ^ 1;
     return Q4_OK;
+}
+
+static void step_free(q4_step* st) {
+    if (st->exec) cudaGraphExecDestroy(st->exec);
+    if (st->capture) cudaStreamDestroy(st->capture);
+    delete st;
+}
+
+q4_status q4_step_create(const q4_linear* linears, int64_t n, q4_step** step) {
+    if (!step) return Q4_ERR_NULL;
+    *step = nullptr;
+    if (!linears) return Q4_ERR_NULL;
+    if (n < 1) return Q4_ERR_SHAPE;
+    for (int64_t i = 0; i < n; ++i) {
+        const q4_linear& l = linears[i];
+        bool empty;
+        const q4_status st = check_matmul(l.codes, l.scales, l.codebook, l.x, l.y, l.M, l.N, l.K, &empty);
+        if (st != Q4_OK) return st;
+    }
+    DeviceInfo dev;
+    q4_status st = gate(&dev);
+    if (st != Q4_OK) return st;
+    q4_step* r = new q4_step();
+    r->device = dev.device;
+    cudaError_t e = cudaStreamCreateWithFlags(&r->capture, cudaStreamNonBlocking);
+    // relaxed: the launchers may set a kernel's shared-memory attribute the
+    // first time they see it, which is not a stream operation
+    if (e == cudaSuccess) e = cudaStreamBeginCapture(r->capture, cudaStreamCaptureModeRelaxed);
+    if (e != cudaSuccess) {
+        step_free(r);
+        return cuda_fail(e);
+    }
+    for (int64_t i = 0; i < n && st == Q4_OK; ++i) {
+        const q4_linear& l = linears[i];
+        if (l.M == 0 || l.N == 0) continue;
+        st = gemm_dispatch(l.codes, l.scales, l.codebook, l.x, l.y, l.M, l.N, l.K, r->capture, dev);
+    }
+    cudaGraph_t graph = nullptr;
+    e = cudaStreamEndCapture(r->capture, &graph);
+    if (st == Q4_OK && e != cudaSuccess) st = cuda_fail(e);
+    if (st == Q4_OK) {
+        e = cudaGraphInstantiate(&r->exec, graph, 0);
+        if (e != cudaSuccess) st = cuda_fail(e);
+    }
+    if (graph) cudaGraphDestroy(graph);
+    if (st != Q4_OK) {
+        step_free(r);
+        return st;
+    }
+    *step = r;
+    return Q4_OK;
+}
+
+q4_status q4_step_launch(q4_step* step, q4_stream_t stream) {
+    if (!step) return Q4_ERR_NULL;
+    const cudaError_t e = cudaGraphLaunch(step->exec, stream);
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
+}
+
+q4_status q4_step_destroy(q4_step* step) {
+    if (!step) return Q4_ERR_NULL;
+    step_free(step);
+    return Q4_OK;
+}
+
+q4_status q4_wait_selftest(uint32_t limit_us, int arrive, uint32_t* waited_us) {
+    if (!waited_us) return Q4_ERR_NULL;
+    *waited_us = 0;
+    if (limit_us < 1 || limit_us > 1000000u) return Q4_ERR_SHAPE;
+    DeviceInfo dev;
+    const q4_status st = gate(&dev);
+    if (st != Q4_OK) return st;
+    const cudaError_t e = run_wait_selftest(limit_us, arrive, waited_us);
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
 }
 
 const char* q4_status_string(q4_status status) {

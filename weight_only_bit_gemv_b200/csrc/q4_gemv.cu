@@ -3,8 +3,8 @@
 // What it computes: y[m][n] = sum_g scale[n][g] * sum_{k in g} cb[code(n,k)] * x[m][k]
 // ("deep-fold", "Method": 64-weight groups with four-bit codes and one FP16
 // scale; the decode GEMV rebuilds values while it multiplies and never writes
-// a dense matrix; "Trapetum" overview: the kernel reads straight out of the
-// codebook).
+// a dense matrix; "Trapetum" overview, "What it does": the kernel decodes
+// each weight from the codebook as it multiplies).
 //
 // Design (HBM-bound: 0.53125 bytes per weight must stream at full bandwidth):
 //  * Code bytes are decoded through a 256-entry byte -> half2 table in shared

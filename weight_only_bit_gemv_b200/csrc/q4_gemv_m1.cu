@@ -669,6 +669,36 @@ cudaError_t launch_variant(const M1& p, int grid, int smem, int slot, cudaStream
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// q4_wait_selftest: the bounded wait above, made to run out on purpose with
+// nothing in flight (no copy, no tensor-memory allocation): one thread waits
+// on an mbarrier that expects one arrival and gets it only if `arrive`.
+// ---------------------------------------------------------------------------
+__device__ unsigned long long g_selftest_waited_ns;
+
+__global__ void wait_selftest_kernel(unsigned long long limit_ns, int arrive) {
+    __shared__ __align__(8) unsigned long long bar_storage;
+    if (threadIdx.x != 0) return;
+    const uint32_t bar = smem_u32(&bar_storage);
+    mbar_init(bar, 1);
+    fence_mbar_init();
+    if (arrive) mbar_arrive(bar);
+    const unsigned long long t0 = globaltimer_ns();
+    const bool ok = mbar_wait(bar, 0u, limit_ns);
+    g_selftest_waited_ns = globaltimer_ns() - t0;
+    if (!ok) atomicOr(&g_gemv_m1_error, 0x80u);
+}
+
+cudaError_t run_wait_selftest(uint32_t limit_us, int arrive, uint32_t* waited_us) {
+    wait_selftest_kernel<<<1, 32>>>(static_cast<unsigned long long>(limit_us) * 1000ull, arrive);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    unsigned long long ns = 0;
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&ns, g_selftest_waited_ns, sizeof(ns));
+    if (e == cudaSuccess) *waited_us = static_cast<uint32_t>(ns / 1000ull);
+    return e;
+}
+
 cudaError_t take_gemv_m1_error(unsigned int* out) {
     unsigned int zero = 0;
     cudaError_t e = cudaMemcpyFromSymbol(out, g_gemv_m1_error, sizeof(unsigned int));

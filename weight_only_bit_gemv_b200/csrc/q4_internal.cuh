@@ -81,6 +81,10 @@ cudaError_t launch_gemv2(const uint8_t* codes, const uint16_t* scales, const uin
                          const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
                          const DeviceInfo& dev);
 
+// q4_wait_selftest's kernel (q4_gemv_m1.cu): a bounded mbarrier wait of at
+// most limit_us that runs out unless `arrive`; synchronizes the device.
+cudaError_t run_wait_selftest(uint32_t limit_us, int arrive, uint32_t* waited_us);
+
 // Copy out and clear the timeout bits that a kernel family's bounded waits
 // set (synchronous; see q4_timeout_flags).
 cudaError_t take_gemv_m1_error(unsigned int* out);
