@@ -284,10 +284,13 @@ int q4_abi_version(void);
  * smallest magnitude); bit-identical to a serial IEEE implementation.
  * q4_gemv2: one token, y[n] = sum_k W[n][k] * x[k], x [K] bfloat16, y [N]
  * fp32.  Products are exact (x rounded to binary16, as q4_gemv), the sums
- * fp32.  y is zeroed on the stream and then accumulated by several CTAs, so
- * the order of the fp32 additions is not fixed from run to run.
+ * fp32.  Up to K = 57344 each element of y is written once by one thread
+ * block (programmatic dependent launch, as q4_gemv), so the result does not
+ * depend on timing; above that, y is zeroed on the stream and then
+ * accumulated by several thread blocks, so the order of the fp32 additions
+ * is not fixed from run to run.
  * Validation as q4_dequant / q4_gemv (M = 1 implied), plus Q4_ERR_SHAPE for
- * K > Q4_GEMV2_MAX_K (x is staged in shared memory, 136 bytes per group).
+ * K > Q4_GEMV2_MAX_K (x is staged in shared memory).
  */
 #define Q4_GEMV2_MAX_K 98304
 q4_status q4_pack2(const float* w, const uint16_t* codebook4, uint8_t* codes,
@@ -363,8 +366,9 @@ q4_status q4_wait_selftest(uint32_t limit_us, int arrive, uint32_t* waited_us);
  * a device word, the kernel drains what it has in flight, frees its tensor
  * memory and exits, leaving its output incomplete.  This call synchronizes the
  * current device, stores the bits set since the last call in *flags and
- * clears them: bits 0-11 the M = 1 GEMV (bit 7: q4_wait_selftest's wait ran
- * out; bit 8: its shared-memory layout did not match the device; bits 9-11:
+ * clears them: bits 1-3 the two-bit GEMV (producer, drain and consumer
+ * waits), bits 4-11 the M = 1 GEMV (bit 7: q4_wait_selftest's wait ran out;
+ * bit 8: its shared-memory layout did not match the device; bits 9-11:
  * producer, drain and consumer waits), bits
  * 12-15 the M = 2..24 kernel (the same four conditions), bits 16-31 the
  * tensor-core GEMM (M > 24); 0 = none.  Not an operation of the method; a

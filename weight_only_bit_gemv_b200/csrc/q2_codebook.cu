@@ -27,6 +27,7 @@
 // cut into equal contiguous ranges, one per warp; a warp adds each finished
 // tile's sums into y with red.add (y is zeroed first on the same stream).
 #include "q4_internal.cuh"
+#include "q4_sm100.cuh"
 
 namespace q4 {
 namespace {
@@ -299,7 +300,515 @@ __global__ void __launch_bounds__(kQ2Threads, 2)
     flush(cur_rt);
 }
 
+// ---------------------------------------------------------------------------
+// gemv2 on a bulk-copy ring (the path for K <= kR2MaxK)
+// ---------------------------------------------------------------------------
+// Weight stream: CTA c owns the rows [N c / grid, N (c + 1) / grid); a
+// producer warp copies 16-row tiles of their codes into a shared-memory ring
+// with 1-D bulk copies (one contiguous copy per tile when a row is at most
+// 2 KB, else one ~2 KB segment per row per stage), and the stage's scales
+// with cp.async beside them; both complete on the stage's mbarrier.
+//
+// Consumer warp w takes unit w of every stage: 16 rows x 128 code bytes
+// (8 groups, 512 k).  Lane (g, tq) reads 32 bytes of rows g and g + 8: group
+// 2 tq ("lo") and group 2 tq + 1 ("hi") of the unit.  MMA (q, i, h), 32 per
+// unit, takes from word q of each of those four 16-byte groups the codes at
+// bit position 2 i of bytes 2 h and 2 h + 1, i.e. k = 16 q + 8 h + 4 e + i
+// (e = 0, 1) of the group, rebuilt by one PRMT each from the codebook held as
+// split low and high bytes; the selector of four codes is
+// (word & (3 << 2 i) per byte) * 0x11 >> 2 i + 0x40 per byte (one LOP and
+// one IMAD).  a0 / a2 carry row g's lo / hi group, a1 / a3 row g + 8's.
+//
+// Groups as B columns: B column n holds x of the unit's group n and zeros
+// elsewhere, so the accumulator column n is group n's partial sum and lane
+// (g, tq) holds exactly its own two groups (columns 2 tq, 2 tq + 1) of rows g
+// and g + 8, which it scales in fp32 with those groups' scales.  In the B
+// fragment only lane (2 tq, tq) has a nonzero b0 and lane (2 tq + 1, tq) a
+// nonzero b1: every lane holds the binary16 x of group g of its unit and
+// multiplies it by a per-lane 1.0 / 0.0 half2 mask (HMUL2, on the FMA pipe)
+// into b0 and b1.  Products are exact and sums fp32, as in q4_gemv.
+//
+// A warp keeps its units' sums of a tile in its own shared-memory slot; at
+// the end of a pass of tiles the CTA adds the slots and writes each y element
+// once (no memset, no atomics).  Programmatic dependent launch as q4_gemv.
+constexpr int kR2CW = 16;                      // consumer warps
+constexpr int kR2Threads = (kR2CW + 1) * 32;   // + one producer warp
+constexpr int kR2Unit = 128;                   // code bytes of a row per unit
+constexpr int kR2MaxKC = 2048;                 // code bytes of a row per stage
+constexpr int kR2MaxStages = 6;
+constexpr int kR2MinPassTiles = 4;
+constexpr int kR2MaxPassTiles = 64;
+constexpr uint32_t kR2TileSlotBytes = kR2CW * 16 * 4;
+
+__device__ unsigned int g_gemv2_error;
+
+// Multipliers of the selector arithmetic, passed as kernel arguments so that
+// they stay integer multiplies (the FMA pipe) instead of being folded into
+// shifts and adds (the ALU pipe, which the PRMTs already keep busy).
+struct SelMul {
+    uint32_t k11;      // 0x11: c -> c | c << 4 in each byte
+    uint32_t k11_16;   // 0x11 << 16: the same, bytes 2 and 3 moved down by 16
+    uint32_t k11_26;   // 0x11 << 26: codes at bits 6-7 of each byte, moved down by 6
+    uint32_t k11_10;   // 0x11 << 10: the same, moved down by 22
+    uint32_t sh30, sh28;  // 2^30, 2^28: mul.hi by them shifts right by 2, 4
+};
+
+struct G2 {
+    const uint8_t* codes;
+    const uint16_t* scales;
+    const uint16_t* cb;
+    const uint16_t* x;
+    float* y;
+    int N, K, G;
+    int R;      // code bytes of a row (K / 4)
+    int KC;     // code bytes of a row per stage (the ring's row pitch)
+    int GS;     // groups of a row per stage (KC / 16)
+    int C;      // stages per 16-row tile
+    int NS;     // ring stages
+    int PT;     // tiles per pass of the partial slots
+    int units;  // units of a row (ceil(R / 128))
+    uint32_t bar_off, x_off, zero_off, ring_off, stage_bytes, scale_off;
+    SelMul k;
+};
+
+__device__ __forceinline__ uint4 lds128_v(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t word4(const uint4& v, int q) {
+    return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
+}
+
+__device__ __forceinline__ uint32_t mulhi(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.hi.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t madhi(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t madlo(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// PRMT selectors for the four codes at bit position 2 i of the bytes of w:
+// the low 16 bits of *s0 pick bytes 0 and 1, those of *s1 bytes 2 and 3, as
+// (cb[c] low byte, cb[c] high byte) pairs; PRMT nibble c picks the
+// codebook's low byte of entry c, 4 + c its high byte, so a code c becomes the
+// selector byte c * 0x11 + 0x40.  Each product stays inside its byte or is
+// moved whole by the high half of the product, so no byte carries into the
+// next.
+template <int kI>
+__device__ __forceinline__ void selectors(uint32_t w, const SelMul& k, uint32_t* s0, uint32_t* s1) {
+    uint32_t t;
+    if constexpr (kI == 0) {
+        t = w & 0x03030303u;
+    } else if constexpr (kI == 3) {
+        t = w & 0xC0C0C0C0u;
+    } else {
+        t = mulhi(w, kI == 1 ? k.sh30 : k.sh28) & 0x03030303u;  // codes moved to bits 0-1
+    }
+    if constexpr (kI == 3) {
+        *s0 = madhi(t, k.k11_26, 0x40404040u);
+        *s1 = madhi(t, k.k11_10, 0x4040u);
+    } else {
+        *s0 = madlo(t, k.k11, 0x40404040u);
+        *s1 = madhi(t, k.k11_16, 0x4040u);
+    }
+}
+
+// binary16 pair (lo, hi) from two bfloat16 values
+__device__ __forceinline__ uint32_t bf16pair_to_f16x2(uint32_t lo, uint32_t hi) {
+    const __half2 h = __floats2half2_rn(__uint_as_float(lo << 16), __uint_as_float(hi << 16));
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int kSW>
+__device__ __forceinline__ void copy_scales(uint32_t dst, const uint16_t* src) {
+    if (kSW == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+    else if (kSW == 8)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+    else if (kSW == 4)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+    else
+        sts_u16(dst, __ldg(reinterpret_cast<const unsigned short*>(src)));
+}
+
+// kWhole: a tile is one stage (rows of at most 2 KB); kSW: bytes per scale
+// copy (16, 8, 4 with cp.async; 2 = plain loads, for an odd group count).
+template <bool kWhole, int kSW>
+__global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int g = lane >> 2, tq = lane & 3;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bars = base + p.bar_off;
+    const int NS = p.NS;
+    const int r0 = static_cast<int>(static_cast<int64_t>(p.N) * blockIdx.x / gridDim.x);
+    const int r1 = static_cast<int>(static_cast<int64_t>(p.N) * (blockIdx.x + 1) / gridDim.x);
+    const int nrows = r1 - r0;
+    const int T = (nrows + 15) >> 4;
+    const int total = T * p.C;
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(bars + 8u * s, 33);             // expect_tx + the producer lanes' scale copies
+            mbar_init(bars + 8u * (NS + s), kR2CW);   // one arrival per consumer warp
+        }
+        fence_mbar_init();
+    }
+    // warm L2 with the first tile, its scales and x while the preceding kernel finishes
+    if (warp == kR2CW && total > 0) {
+        const int rows = min(16, nrows);
+        if (kWhole) {
+            if (lane == 0)
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.codes + static_cast<int64_t>(r0) * p.R),
+                             "r"(static_cast<uint32_t>(rows * p.R)) : "memory");
+        } else if (lane < rows) {
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.codes + static_cast<int64_t>(r0 + lane) * p.R),
+                         "r"(static_cast<uint32_t>(min(p.KC, p.R))) : "memory");
+        }
+        if (lane == 31)
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p.x), "r"(static_cast<uint32_t>(p.K) * 2u)
+                         : "memory");
+    }
+    __syncthreads();
+
+    if (warp == kR2CW) {
+        // ------------------------------ producer ------------------------------
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        int slot = 0, t = 0, c = 0;
+        uint32_t eparity = 1;
+        int issued = 0;
+        for (int i = 0; i < total; ++i) {
+            if (i >= NS) {
+                uint32_t ok = 1;
+                if (lane == 0) ok = mbar_wait(bars + 8u * (NS + slot), eparity) ? 1u : 0u;
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) {
+                    if (lane == 0) atomicOr(&g_gemv2_error, 0x2u);
+                    break;
+                }
+            }
+            const int rows = min(16, nrows - 16 * t);
+            const int row0 = r0 + 16 * t;
+            const uint32_t dst = base + p.ring_off + slot * p.stage_bytes;
+            const uint32_t full = bars + 8u * slot;
+            const int cbytes = kWhole ? p.R : min(p.KC, p.R - c * p.KC);
+            if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(rows * cbytes));
+            __syncwarp();
+            if (kWhole) {
+                if (lane == 0)
+                    bulk_load(dst, p.codes + static_cast<int64_t>(row0) * p.R, static_cast<uint32_t>(rows * p.R), full);
+            } else if (lane < rows) {
+                bulk_load(dst + lane * p.KC, p.codes + static_cast<int64_t>(row0 + lane) * p.R + c * p.KC,
+                          static_cast<uint32_t>(cbytes), full);
+            }
+            // scales of the stage: rows x ng groups, row pitch GS in the stage
+            const int g0 = kWhole ? 0 : c * p.GS;
+            const int ng = kWhole ? p.G : min(p.GS, p.G - g0);
+            const int per_row = ng * 2 / kSW;
+            const uint32_t sdst = dst + p.scale_off;
+            for (int j = lane; j < rows * per_row; j += 32) {
+                const int r = j / per_row, q = j - r * per_row;
+                copy_scales<kSW>(sdst + r * (p.GS * 2) + q * kSW,
+                                 p.scales + static_cast<int64_t>(row0 + r) * p.G + g0 + q * (kSW / 2));
+            }
+            if (kSW > 2)
+                asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(full) : "memory");
+            else
+                mbar_arrive(full);
+            ++issued;
+            if (++c == p.C) {
+                c = 0;
+                ++t;
+            }
+            if (++slot == NS) {
+                slot = 0;
+                eparity ^= 1u;
+            }
+        }
+        // leave only once this warp's copies have landed (bounded)
+        if (lane == 0) {
+            for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i)
+                if (!mbar_wait(bars + 8u * (i % NS), (i / NS) & 1)) {
+                    atomicOr(&g_gemv2_error, 0x4u);
+                    break;
+                }
+        }
+        return;
+    }
+
+    // ------------------------------- consumers ------------------------------
+    float* acc_s = reinterpret_cast<float*>(smem);  // [PT tiles][kR2CW warps][16 rows]
+    const int upk = kWhole ? p.units : p.KC / kR2Unit;
+    const uint32_t off1 = 32 * tq + 16 * (g & 1), off2 = 32 * tq + 16 * (1 - (g & 1));
+    const bool swap = (g & 1) != 0;
+    const uint32_t rowA = static_cast<uint32_t>(g * p.KC), rowB = static_cast<uint32_t>((g + 8) * p.KC);
+    // B operand: b0 carries x for lane (2 tq, tq) and b1 for lane (2 tq + 1,
+    // tq); every other b register reads the zero block
+    const bool act0 = g == 2 * tq, act1 = g == 2 * tq + 1;
+    const SelMul km = p.k;
+
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    uint32_t cbl = 0, cbh = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const uint32_t hv = __ldg(p.cb + e);
+        cbl |= (hv & 0xFFu) << (8 * e);
+        cbh |= (hv >> 8) << (8 * e);
+    }
+    {
+        // x of every unit as binary16 in MMA order: MMA m = 8 q + 2 i + h of
+        // group 8 u + a holds (x[16 q + 8 h + i], x[16 q + 8 h + 4 + i]) of the
+        // group, at x_off + 1024 u + 128 (m / 4) + 16 a + 4 (m % 4); zeros
+        // past the last group
+        const int items = p.units * 8 * 8;  // (unit, a, q, h)
+        for (int it = tid; it < items; it += kR2CW * 32) {
+            const int h = it & 1, q = (it >> 1) & 3, a = (it >> 3) & 7, u = it >> 6;
+            const int grp = 8 * u + a;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (grp < p.G)
+                v = __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(grp) * kGroup + 16 * q + 8 * h));
+            const uint32_t e[8] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16,
+                                   v.z & 0xFFFFu, v.z >> 16, v.w & 0xFFFFu, v.w >> 16};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int m = 8 * q + 2 * i + h;
+                *reinterpret_cast<uint32_t*>(smem + p.x_off + 1024 * u + 128 * (m >> 2) + 16 * a + 4 * (m & 3)) =
+                    bf16pair_to_f16x2(e[i], e[4 + i]);
+            }
+        }
+        for (int it = tid; it < 1024 / 16; it += kR2CW * 32)
+            *reinterpret_cast<uint4*>(smem + p.zero_off + 16 * it) = make_uint4(0u, 0u, 0u, 0u);
+        asm volatile("bar.sync 1, %0;" ::"n"(kR2CW * 32) : "memory");
+    }
+
+    bool bad = false;
+    int slot = 0;
+    uint32_t fparity = 0;
+    for (int pt0 = 0; pt0 < T; pt0 += p.PT) {
+        const int pt1 = min(T, pt0 + p.PT);
+        for (int t = pt0; t < pt1; ++t) {
+            float acc_g = 0.f, acc_h = 0.f;  // rows g and g + 8
+            for (int c = 0; c < p.C; ++c) {
+                if (!bad && !mbar_wait(bars + 8u * slot, fparity)) {
+                    bad = true;
+                    if (lane == 0) atomicOr(&g_gemv2_error, 0x8u);
+                }
+                const int U = c * upk + warp;  // unit of the row
+                if (!bad && warp < upk && U < p.units) {
+                    const uint32_t sb = base + p.ring_off + slot * p.stage_bytes;
+                    // x of group 8 U + g for the active lanes, the zero block for the rest
+                    const uint32_t xg = base + p.x_off + 1024 * U + 16 * g, xz = base + p.zero_off;
+                    const uint32_t xa0 = act0 ? xg : xz, xa1 = act1 ? xg : xz;
+                    const uint32_t ua = sb + warp * kR2Unit;
+                    const uint4 a1 = lds128_v(ua + rowA + off1), a2 = lds128_v(ua + rowA + off2);
+                    const uint4 b1 = lds128_v(ua + rowB + off1), b2 = lds128_v(ua + rowB + off2);
+                    const uint4 lo_g = swap ? a2 : a1, hi_g = swap ? a1 : a2;
+                    const uint4 lo_h = swap ? b2 : b1, hi_h = swap ? b1 : b2;
+                    float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 xv0 = lds128_v(xa0 + 256 * q), xv1 = lds128_v(xa0 + 256 * q + 128);
+                        const uint4 xw0 = lds128_v(xa1 + 256 * q), xw1 = lds128_v(xa1 + 256 * q + 128);
+                        const uint32_t xb0[8] = {xv0.x, xv0.y, xv0.z, xv0.w, xv1.x, xv1.y, xv1.z, xv1.w};
+                        const uint32_t xb1[8] = {xw0.x, xw0.y, xw0.z, xw0.w, xw1.x, xw1.y, xw1.z, xw1.w};
+                        const uint32_t wlg = word4(lo_g, q), whg = word4(hi_g, q);
+                        const uint32_t wlh = word4(lo_h, q), whh = word4(hi_h, q);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            uint32_t slg0, slg1, shg0, shg1, slh0, slh1, shh0, shh1;
+                            switch (i) {
+                                case 0:
+                                    selectors<0>(wlg, km, &slg0, &slg1); selectors<0>(whg, km, &shg0, &shg1);
+                                    selectors<0>(wlh, km, &slh0, &slh1); selectors<0>(whh, km, &shh0, &shh1);
+                                    break;
+                                case 1:
+                                    selectors<1>(wlg, km, &slg0, &slg1); selectors<1>(whg, km, &shg0, &shg1);
+                                    selectors<1>(wlh, km, &slh0, &slh1); selectors<1>(whh, km, &shh0, &shh1);
+                                    break;
+                                case 2:
+                                    selectors<2>(wlg, km, &slg0, &slg1); selectors<2>(whg, km, &shg0, &shg1);
+                                    selectors<2>(wlh, km, &slh0, &slh1); selectors<2>(whh, km, &shh0, &shh1);
+                                    break;
+                                default:
+                                    selectors<3>(wlg, km, &slg0, &slg1); selectors<3>(whg, km, &shg0, &shg1);
+                                    selectors<3>(wlh, km, &slh0, &slh1); selectors<3>(whh, km, &shh0, &shh1);
+                                    break;
+                            }
+                            uint32_t a[4];
+                            a[0] = __byte_perm(cbl, cbh, slg0);
+                            a[1] = __byte_perm(cbl, cbh, slh0);
+                            a[2] = __byte_perm(cbl, cbh, shg0);
+                            a[3] = __byte_perm(cbl, cbh, shh0);
+                            mma_16816(d0, a, xb0[2 * i], xb1[2 * i], d0);
+                            a[0] = __byte_perm(cbl, cbh, slg1);
+                            a[1] = __byte_perm(cbl, cbh, slh1);
+                            a[2] = __byte_perm(cbl, cbh, shg1);
+                            a[3] = __byte_perm(cbl, cbh, shh1);
+                            mma_16816(d1, a, xb0[2 * i + 1], xb1[2 * i + 1], d1);
+                        }
+                    }
+                    // columns 2 tq, 2 tq + 1: this lane's groups of rows g, g + 8
+                    const int gl = warp * 8 + 2 * tq;  // group index within the stage's scale rows
+                    const int ga = U * 8 + 2 * tq;      // group index within the row
+                    const uint32_t srow_g = sb + p.scale_off + g * (p.GS * 2) + 2 * gl;
+                    const uint32_t srow_h = srow_g + 8 * (p.GS * 2);
+                    float s00 = 0.f, s01 = 0.f, s10 = 0.f, s11 = 0.f;
+                    if (ga < p.G) {
+                        s00 = __half2float(__ushort_as_half(ld_smem<uint16_t>(smem, srow_g - base)));
+                        s10 = __half2float(__ushort_as_half(ld_smem<uint16_t>(smem, srow_h - base)));
+                    }
+                    if (ga + 1 < p.G) {
+                        s01 = __half2float(__ushort_as_half(ld_smem<uint16_t>(smem, srow_g - base + 2)));
+                        s11 = __half2float(__ushort_as_half(ld_smem<uint16_t>(smem, srow_h - base + 2)));
+                    }
+                    acc_g = fmaf(s00, d0[0] + d1[0], acc_g);
+                    acc_g = fmaf(s01, d0[1] + d1[1], acc_g);
+                    acc_h = fmaf(s10, d0[2] + d1[2], acc_h);
+                    acc_h = fmaf(s11, d0[3] + d1[3], acc_h);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + 8u * (NS + slot));
+                if (++slot == NS) {
+                    slot = 0;
+                    fparity ^= 1u;
+                }
+            }
+            // the four lanes of a row hold its eight groups' sums
+            acc_g += __shfl_xor_sync(0xFFFFFFFFu, acc_g, 1);
+            acc_g += __shfl_xor_sync(0xFFFFFFFFu, acc_g, 2);
+            acc_h += __shfl_xor_sync(0xFFFFFFFFu, acc_h, 1);
+            acc_h += __shfl_xor_sync(0xFFFFFFFFu, acc_h, 2);
+            if (tq == 0) {
+                float* slot_w = acc_s + ((t - pt0) * kR2CW + warp) * 16;
+                slot_w[g] = acc_g;
+                slot_w[g + 8] = acc_h;
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kR2CW * 32) : "memory");
+        const int row_end = min(nrows, 16 * pt1);
+        for (int r = 16 * pt0 + tid; r < row_end; r += kR2CW * 32) {
+            const int rl = r - 16 * pt0;
+            const float* q = acc_s + (rl >> 4) * kR2CW * 16 + (rl & 15);
+            float sum = 0.f;
+#pragma unroll
+            for (int w = 0; w < kR2CW; ++w) sum += q[16 * w];
+            p.y[r0 + r] = sum;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kR2CW * 32) : "memory");
+    }
+}
+
+template <bool kWhole, int kSW>
+cudaError_t launch_ring2(const G2& p, int grid, int smem, int slot, cudaStream_t s, const DeviceInfo& dev) {
+    auto kern = gemv2_ring_kernel<kWhole, kSW>;
+    cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem, slot, dev.device);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kR2Threads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+// Plans and launches the ring kernel; cudaErrorNotSupported when the shape
+// does not fit its shared-memory layout (x of a long row plus the ring).
+cudaError_t launch_gemv2_ring(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
+                              const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
+                              const DeviceInfo& dev) {
+    G2 p{};
+    p.codes = codes;
+    p.scales = scales;
+    p.cb = cb;
+    p.x = x;
+    p.y = y;
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.G = static_cast<int>(K / kGroup);
+    p.R = static_cast<int>(K / 4);
+    p.k = SelMul{0x11u, 0x11u << 16, 0x11u << 26, 0x11u << 10, 1u << 30, 1u << 28};
+    p.units = (p.R + kR2Unit - 1) / kR2Unit;
+    const bool whole = p.R <= kR2MaxKC;
+    if (whole) {
+        p.C = 1;
+        p.KC = p.R;
+        p.GS = p.G;
+    } else {
+        p.C = (p.R + kR2MaxKC - 1) / kR2MaxKC;
+        p.KC = ((p.R + p.C - 1) / p.C + kR2Unit - 1) / kR2Unit * kR2Unit;
+        p.C = (p.R + p.KC - 1) / p.KC;
+        p.GS = p.KC / 16;
+    }
+    const uint32_t code_bytes = (static_cast<uint32_t>(16 * p.KC) + 127u) & ~127u;
+    p.scale_off = code_bytes;
+    p.stage_bytes = code_bytes + ((static_cast<uint32_t>(16 * p.GS * 2) + 127u) & ~127u);
+    const uint32_t x_bytes = static_cast<uint32_t>(p.units) * 1024u;
+    auto layout = [&](int pt) {
+        p.PT = pt;
+        p.bar_off = static_cast<uint32_t>(pt) * kR2TileSlotBytes;
+        p.zero_off = p.bar_off + 128u;
+        p.x_off = p.zero_off + 1024u;
+        p.ring_off = (p.x_off + x_bytes + 127u) & ~127u;
+        return dev.smem_optin - static_cast<int>(p.ring_off);
+    };
+    int ns = layout(kR2MinPassTiles) / static_cast<int>(p.stage_bytes);
+    if (ns > kR2MaxStages) ns = kR2MaxStages;
+    if (ns < 2) return cudaErrorNotSupported;
+    p.NS = ns;
+    const int64_t tiles_per_cta = ((N + dev.sm_count - 1) / dev.sm_count + 15) / 16 + 1;
+    const int pt_cap = static_cast<int>(tiles_per_cta < kR2MaxPassTiles ? tiles_per_cta : kR2MaxPassTiles);
+    int pt = pt_cap < kR2MinPassTiles ? kR2MinPassTiles : pt_cap;
+    while (pt > kR2MinPassTiles && layout(pt) < ns * static_cast<int>(p.stage_bytes)) --pt;
+    layout(pt);
+    const int smem = static_cast<int>(p.ring_off + ns * p.stage_bytes);
+    if (smem > dev.smem_optin) return cudaErrorNotSupported;
+    const int64_t tiles = (N + 15) / 16;
+    const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+    // widest scale copy that every source and destination offset allows
+    const int gcd_groups = p.G % 8 == 0 && p.GS % 8 == 0 ? 8 : (p.G % 4 == 0 && p.GS % 4 == 0 ? 4 : (p.G % 2 == 0 && p.GS % 2 == 0 ? 2 : 1));
+    if (whole) {
+        switch (gcd_groups) {
+            case 8: return launch_ring2<true, 16>(p, grid, smem, 51, s, dev);
+            case 4: return launch_ring2<true, 8>(p, grid, smem, 52, s, dev);
+            case 2: return launch_ring2<true, 4>(p, grid, smem, 53, s, dev);
+            default: return launch_ring2<true, 2>(p, grid, smem, 54, s, dev);
+        }
+    }
+    switch (gcd_groups) {
+        case 8: return launch_ring2<false, 16>(p, grid, smem, 55, s, dev);
+        case 4: return launch_ring2<false, 8>(p, grid, smem, 56, s, dev);
+        case 2: return launch_ring2<false, 4>(p, grid, smem, 57, s, dev);
+        default: return launch_ring2<false, 2>(p, grid, smem, 58, s, dev);
+    }
+}
+
 }  // namespace
+
+cudaError_t take_gemv2_error(unsigned int* out) {
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_gemv2_error, sizeof(unsigned int));
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_gemv2_error, &zero, sizeof(unsigned int));
+    return e;
+}
 
 cudaError_t launch_pack2(const float* w, const uint16_t* cb, uint8_t* codes, uint16_t* scales,
                          int64_t N, int64_t K, cudaStream_t s, const DeviceInfo& dev) {
@@ -320,6 +829,13 @@ int gemv2_smem_bytes(int64_t K) { return static_cast<int>((K / kGroup) * kQ2XGro
 cudaError_t launch_gemv2(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                          const uint16_t* x, float* y, int64_t N, int64_t K, cudaStream_t s,
                          const DeviceInfo& dev) {
+    if (dev.smem_optin >= 64 * 1024) {
+        const cudaError_t r = launch_gemv2_ring(codes, scales, cb, x, y, N, K, s, dev);
+        if (r != cudaErrorNotSupported) return r;
+        (void)cudaGetLastError();
+    }
+    // rows too long for the ring's shared-memory layout: per-lane loads, y
+    // zeroed and then added into
     const int smem = gemv2_smem_bytes(K);
     if (smem > dev.smem_optin) return cudaErrorNotSupported;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(gemv2_kernel), smem, 50, dev.device);

@@ -475,12 +475,13 @@ q4_status q4_gemv2(const uint8_t* codes, const uint16_t* scales, const uint16_t*
 q4_status q4_timeout_flags(uint32_t* flags) {
     if (!flags) return Q4_ERR_NULL;
     *flags = 0;
-    unsigned int a = 0, b = 0, c = 0;
+    unsigned int a = 0, b = 0, c = 0, d = 0;
     cudaError_t e = take_gemv_m1_error(&a);
     if (e == cudaSuccess) e = take_gemm_tc_error(&b);
     if (e == cudaSuccess) e = take_gemm_small_error(&c);
+    if (e == cudaSuccess) e = take_gemv2_error(&d);
     if (e != cudaSuccess) return cuda_fail(e);
-    *flags = (a & 0x0FFFu) | ((c & 0x0F00u) << 4) | ((b & 0xFFFFu) << 16);
+    *flags = (a & 0x0FF0u) | (d & 0x000Eu) | ((c & 0x0F00u) << 4) | ((b & 0xFFFFu) << 16);
     return Q4_OK;
 }
 

@@ -90,6 +90,7 @@ cudaError_t run_wait_selftest(uint32_t limit_us, int arrive, uint32_t* waited_us
 cudaError_t take_gemv_m1_error(unsigned int* out);
 cudaError_t take_gemm_tc_error(unsigned int* out);
 cudaError_t take_gemm_small_error(unsigned int* out);
+cudaError_t take_gemv2_error(unsigned int* out);
 
 // ---------------------------------------------------------------------------
 // device helpers
