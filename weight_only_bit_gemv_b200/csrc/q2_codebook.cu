@@ -342,15 +342,12 @@ constexpr uint32_t kR2TileSlotBytes = kR2CW * 16 * 4;
 
 __device__ unsigned int g_gemv2_error;
 
-// Multipliers of the selector arithmetic, passed as kernel arguments so that
-// they stay integer multiplies (the FMA pipe) instead of being folded into
-// shifts and adds (the ALU pipe, which the PRMTs already keep busy).
+// The multiplier of the selector arithmetic (0x11) is passed as a kernel
+// argument so that it stays one integer multiply-add (the FMA pipe) instead of
+// being folded into a shift and an add (the ALU pipe, which the PRMTs keep
+// busy).
 struct SelMul {
-    uint32_t k11;      // 0x11: c -> c | c << 4 in each byte
-    uint32_t k11_16;   // 0x11 << 16: the same, bytes 2 and 3 moved down by 16
-    uint32_t k11_26;   // 0x11 << 26: codes at bits 6-7 of each byte, moved down by 6
-    uint32_t k11_10;   // 0x11 << 10: the same, moved down by 22
-    uint32_t sh30, sh28;  // 2^30, 2^28: mul.hi by them shifts right by 2, 4
+    uint32_t k11;  // 0x11: a code c in bits 0-1 of a byte becomes c | c << 4
 };
 
 struct G2 {
@@ -383,16 +380,6 @@ __device__ __forceinline__ uint32_t word4(const uint4& v, int q) {
     return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
 }
 
-__device__ __forceinline__ uint32_t mulhi(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("mul.hi.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-__device__ __forceinline__ uint32_t madhi(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t d;
-    asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
 __device__ __forceinline__ uint32_t madlo(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t d;
     asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
@@ -401,28 +388,17 @@ __device__ __forceinline__ uint32_t madlo(uint32_t a, uint32_t b, uint32_t c) {
 
 // PRMT selectors for the four codes at bit position 2 i of the bytes of w:
 // the low 16 bits of *s0 pick bytes 0 and 1, those of *s1 bytes 2 and 3, as
-// (cb[c] low byte, cb[c] high byte) pairs; PRMT nibble c picks the
-// codebook's low byte of entry c, 4 + c its high byte, so a code c becomes the
-// selector byte c * 0x11 + 0x40.  Each product stays inside its byte or is
-// moved whole by the high half of the product, so no byte carries into the
-// next.
+// (cb[c] low byte, cb[c] high byte) pairs.  PRMT nibble c picks the
+// codebook's low byte of entry c and 4 + c its high byte, so a code c becomes
+// the selector byte c * 0x11 + 0x40; each code is moved to bits 0-1 of its
+// byte first, so no product carries into the next byte.  (Measured on B200:
+// folding the shift into the high half of a product, mad.hi, cost about a
+// quarter more time, as it is not one instruction.)
 template <int kI>
 __device__ __forceinline__ void selectors(uint32_t w, const SelMul& k, uint32_t* s0, uint32_t* s1) {
-    uint32_t t;
-    if constexpr (kI == 0) {
-        t = w & 0x03030303u;
-    } else if constexpr (kI == 3) {
-        t = w & 0xC0C0C0C0u;
-    } else {
-        t = mulhi(w, kI == 1 ? k.sh30 : k.sh28) & 0x03030303u;  // codes moved to bits 0-1
-    }
-    if constexpr (kI == 3) {
-        *s0 = madhi(t, k.k11_26, 0x40404040u);
-        *s1 = madhi(t, k.k11_10, 0x4040u);
-    } else {
-        *s0 = madlo(t, k.k11, 0x40404040u);
-        *s1 = madhi(t, k.k11_16, 0x4040u);
-    }
+    const uint32_t t = (w >> (2 * kI)) & 0x03030303u;
+    *s0 = madlo(t, k.k11, 0x40404040u);
+    *s1 = *s0 >> 16;
 }
 
 // binary16 pair (lo, hi) from two bfloat16 values
@@ -745,7 +721,7 @@ cudaError_t launch_gemv2_ring(const uint8_t* codes, const uint16_t* scales, cons
     p.K = static_cast<int>(K);
     p.G = static_cast<int>(K / kGroup);
     p.R = static_cast<int>(K / 4);
-    p.k = SelMul{0x11u, 0x11u << 16, 0x11u << 26, 0x11u << 10, 1u << 30, 1u << 28};
+    p.k = SelMul{0x11u};
     p.units = (p.R + kR2Unit - 1) / kR2Unit;
     const bool whole = p.R <= kR2MaxKC;
     if (whole) {
