@@ -395,6 +395,14 @@ def run_ours(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(lins, cb, args.cpu_seconds)
+        cpu["coverage"] = cpu_coverage()
+
+    # per-linear launch time as a fixed cost plus bytes over a streaming rate
+    # (least squares over the step's four linears)
+    xb = np.array([algo_bytes(1, L["lin"].N, L["lin"].K) for L in lins], dtype=np.float64)
+    tb = np.array([statistics.median(p) * 1e3 for p in per], dtype=np.float64)  # us
+    slope, fixed = np.polyfit(xb, tb, 1)
+    fit = f"{fixed:.2f} us fixed + bytes at {1e-3 / slope:.0f} GB/s" if slope > 0 else "n/a"
 
     value = aggregate(bytes_step, ms_step, world) / 1e9
     line = {
@@ -421,6 +429,9 @@ def run_ours(args, world, rank, local):
             "per_linear_us": {L["lin"].name: round(per_ms[j] * 1e3, 3) for j, L in enumerate(lins)},
             "per_linear_us_p10_p50_p90": {L["lin"].name: pcts(per[j]) for j, L in enumerate(lins)},
             "decode_tok_s_equiv_32_layers": round(1e3 / (ms_step * 32), 1),
+            "per_linear_us_p10_p50_p90_str": "; ".join(
+                f"{L['lin'].name} " + "/".join(f"{v:.2f}" for v in pcts(per[j])) for j, L in enumerate(lins)),
+            "per_linear_fit": fit,
         },
         "roofline": {
             "kernel": f"q4_gemv gate_up {lins[dom]['lin'].K}->{lins[dom]['lin'].N}",
@@ -449,6 +460,33 @@ def run_ours(args, world, rank, local):
         "gpu_launches": 4 * K,
         "clocks": clk,
     }
+    cfg = line["config"]
+    if gemm is not None:
+        sw = gemm["sweep"]
+        cfg["prefill_llama2_70b_M256_tflops"] = gemm["tflops"]
+        cfg["prefill_llama2_70b_M256_frac_of_bf16_peak"] = gemm["frac_of_bf16_peak"]
+        cfg["prefill_llama2_70b_tflops_M32_128_256_512"] = " / ".join(
+            f"{sw[k]['tflops']:.1f}" for k in sorted(sw, key=lambda k: int(k[2:])))
+        cfg["prefill_llama2_70b_frac_of_roofline_M32_128_256_512"] = " / ".join(
+            f"{sw[k]['frac_of_roofline']:.3f}" for k in sorted(sw, key=lambda k: int(k[2:])))
+    if step8b is not None:
+        cfg["decode_step_llama31_8b_tok_s"] = step8b["tok_s"]
+        cfg["decode_step_llama31_8b_hbm_frac"] = step8b["hbm_frac_of_measured"]
+    if smallm is not None:
+        cfg["verify_llama31_8b_gbs_M2_4_8_16"] = " / ".join(
+            f"{smallm[k]['gbs']:.0f}" for k in ("M=2", "M=4", "M=8", "M=16") if k in smallm)
+        cfg["verify_llama31_8b_hbm_frac_M2_4_8_16"] = " / ".join(
+            f"{smallm[k]['hbm_frac_of_measured']:.3f}" for k in ("M=2", "M=4", "M=8", "M=16") if k in smallm)
+    if two_bit is not None and "gbs" in two_bit:
+        cfg["two_bit_llama2_70b_layer_gbs"] = two_bit["gbs"]
+        cfg["two_bit_llama2_70b_layer_hbm_frac"] = two_bit["hbm_frac_of_measured"]
+    if embed is not None:
+        cfg["embed_rows_gbs"] = embed["gbs"]
+    if ring is not None:
+        cfg["copy_ring_frac_of_h2d_copy"] = ring["frac_of_h2d_copy"]
+    if bf16_base is not None and "decode_llama2_7b_layer_m1" in bf16_base:
+        cfg["torch_bf16_decode_gbs"] = bf16_base["decode_llama2_7b_layer_m1"]["gbs_at_2B_per_weight"]
+        cfg["torch_bf16_prefill_M256_tflops"] = bf16_base["prefill_llama2_70b_layer_m256"]["tflops"]
     if gemm is not None:
         line["gemm_prefill"] = gemm
     if step8b is not None:
@@ -535,8 +573,8 @@ def bench_prefill(dev, cb, stream, tc_peak, hbm_peak, Ms=(32, 128, 256, 512), ma
     return {"workload": f"llama2_70b_prefill layer (4 linears), M={main_M}", "tflops": round(tf, 2),
             "frac_of_bf16_peak": round(tf / tc_peak, 4), "per_linear": m["lin"],
             "sweep": sweep,
-            "timing": "per linear and M: CUDA graph of 4 back-to-back q4_gemm calls (x conversion, "
-                      "y zeroing when K is split, and the tensor-core GEMM), replayed 5 times",
+            "timing": "per linear and M: CUDA graph of 4 back-to-back q4_gemm calls (y zeroing when "
+                      "K is split, and the tensor-core GEMM, which converts x inside), replayed 5 times",
             "note": "no L2 flush: each linear is 37-253 MB of packed weights, read once per launch; "
                     "frac_of_roofline = sum over the linears of max(flop / tensor peak, bytes / HBM "
                     "peak) over the measured time"}
@@ -564,31 +602,26 @@ def bench_decode_step(dev, cb, stream, hbm_peak, reps=20):
         ys.append(torch.empty((1, lin.N), dtype=torch.float32, device=dev))
     torch.cuda.synchronize()
     nbytes = sum(algo_bytes(1, lin.N, lin.K) for _, _, lin in packs)
-    with torch.cuda.stream(stream):
-        for (codes, scales, lin), y in zip(packs, ys):
-            q4.q4_gemv(codes, scales, cb, xs[lin.K], y)
-    stream.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for (codes, scales, lin), y in zip(packs, ys):
-            q4.q4_gemv(codes, scales, cb, xs[lin.K], y)
+    # the library records the 129 launches as one CUDA graph (q4_step_create)
+    step = q4.Step([(codes, scales, cb, xs[lin.K], y) for (codes, scales, lin), y in zip(packs, ys)])
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         for _ in range(3):
-            g.replay()
+            step.launch(stream)
         e0.record()
         for _ in range(reps):
-            g.replay()
+            step.launch(stream)
         e1.record()
     e1.synchronize()
     ms = e0.elapsed_time(e1) / reps
-    del g, packs, xs, ys
+    step.close()
+    del packs, xs, ys
     torch.cuda.empty_cache()
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"workload": "llama31_8b_step: 32 x (qkv 4096->6144, o 4096->4096, gate_up 4096->28672, "
-                        "down 14336->4096) + lm_head 4096->128256, M=1, 129 q4_gemv launches in one "
-                        "CUDA graph",
+                        "down 14336->4096) + lm_head 4096->128256, M=1, 129 q4_gemv launches recorded "
+                        "by q4_step_create as one CUDA graph, replayed by q4_step_launch",
             "bytes_per_step": nbytes, "ms_per_step": round(ms, 4), "tok_s": round(1e3 / ms, 1),
             "gbs": round(gbs, 1), "hbm_frac_of_measured": round(gbs / hbm_peak, 4)}
 
@@ -909,6 +942,53 @@ def cpu_baseline(lins, cb, seconds):
             "sample": f"first {frac:.1%} of the rows of each of the 4 linears (same seeded "
                       f"weights, packed by the oracle), M=1, one pass; {dt:.1f} s single-threaded",
             "host_cpus": os.cpu_count()}
+
+
+def cpu_coverage(seconds_per_case=1.5):
+    """The oracle (as it stands, single-threaded) on a bounded row sample of
+    each workload, with the time of the whole workload extrapolated from the
+    sample (labelled as such).  Packed operands are seeded random codes and
+    scales of the workload's shapes: the oracle's time does not depend on the
+    values.  Samples are sized by a cost model of the oracle's loops (about
+    27 ns per weight to rebuild a row, plus 2.7 ns per weight and token)."""
+    import oracle
+    cbn = synth.codebook()
+    out = {}
+
+    def run(label, seed, N, K, M, extra=None):
+        n = int(min(N, max(16, seconds_per_case / (K * (27e-9 + 2.7e-9 * M)))))
+        codes, scales = synth.tiny_codes_scales(seed, n, K)
+        x = synth.activations(seed + 1, M, K)
+        t = time.perf_counter()
+        oracle.matmul(codes, scales, cbn, x, with_abs=False)
+        dt = time.perf_counter() - t
+        full_s = dt * N / n
+        r = {"sample_rows": n, "rows": N, "M": M, "K": K, "sample_s": round(dt, 3),
+             "ns_per_weight_token": round(dt / (n * K * M) * 1e9, 3),
+             "full_ms_extrapolated": round(full_s * 1e3, 1),
+             "gbs_extrapolated": round(algo_bytes(M, N, K) / full_s / 1e9, 4)}
+        if extra:
+            r.update(extra)
+        out[label] = r
+        return full_s
+
+    lin = synth.WORKLOADS["tiny"].linears[0]
+    run("tiny 256->128 M=1", 7, lin.N, lin.K, 1)
+    wl = synth.WORKLOADS["llama31_8b_step"]
+    layer_s = 0.0
+    for l in wl.linears:
+        s_l = run(f"llama31_8b {l.name} {l.K}->{l.N} M=1", synth.seed_for(wl.index, 0, l.name), l.N, l.K, 1)
+        layer_s += 0.0 if l.name == "lm_head" else s_l
+    head_s = out[f"llama31_8b lm_head 4096->128256 M=1"]["full_ms_extrapolated"] / 1e3
+    out["llama31_8b step (32 layers + lm_head), extrapolated from one layer"] = {
+        "ms_per_step": round((32 * layer_s + head_s) * 1e3, 1),
+        "tok_s": round(1.0 / (32 * layer_s + head_s), 4)}
+    run("small_m_verify o 4096->4096 M=16", 3001, 4096, 4096, 16)
+    run("llama2_70b_prefill o 8192->8192 M=32", 4001, 8192, 8192, 32,
+        {"tflops_extrapolated": None})
+    r = out["llama2_70b_prefill o 8192->8192 M=32"]
+    r["tflops_extrapolated"] = round(2 * 32 * 8192 * 8192 / (r["full_ms_extrapolated"] * 1e-3) / 1e12, 6)
+    return out
 
 
 def run_reference(args, world, rank):

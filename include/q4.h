@@ -29,13 +29,14 @@
  * Ownership.  Every pointer is device memory owned by the caller (PyTorch,
  * cudaMalloc, ...), except the host-side weights of q4_ring_gemm.  The
  * library keeps no pointer after a call returns and holds only a per-device
- * cache of the device's properties.  It allocates in two places: the
- * stream-ordered scratch of the tensor-core path of q4_gemm (M > 24; M =
- * 17..24 only when the M <= 24 kernel declines a shape: 2 * M * K bytes for
- * the binary16 copy of x), taken from a memory pool the library creates once
- * per device and returned to that pool on the same stream before the call
- * returns (the pool keeps the memory it has mapped); and the two device slots
- * of a q4_ring, which the caller creates and destroys explicitly.
+ * cache of the device's properties.  The matmul, pack and dequant calls
+ * allocate nothing at run time.  Two fixed device arrays are part of the
+ * library's image, held by every GPU that loads it until the process exits:
+ * 32 MiB for q4_gemm's binary16 copy of x (see q4_gemm) and 8 MiB for
+ * q4_gemm_noalloc.  The library creates one event per device the first time
+ * q4_gemm takes its tensor-core path there.  Explicitly created objects
+ * allocate what their create call says: the two device slots of a q4_ring,
+ * and the stream and graph of a q4_step.
  * All calls are asynchronous on the caller's stream (0 = legacy default
  * stream); none synchronizes the host except q4_timeout_flags and
  * q4_ring_destroy.  Inputs and outputs must not overlap.  The calls are
@@ -169,8 +170,14 @@ q4_status q4_gemv(const uint8_t* codes, const uint16_t* scales,
  * exact sum per element (for the tensor-core path this holds statistically:
  * the binary16 rounding of W and x is a relative error of at most 2^-11 per
  * term, far inside the bound once K is a few hundred).
- * The tensor-core path first converts x to binary16 into stream-ordered
- * scratch (see Ownership); a failed scratch allocation returns Q4_ERR_CUDA.  When the
+ * The tensor-core path first converts x to binary16 into a fixed 32 MiB
+ * device array (see Ownership), in chunks of tokens when 2 * M * K is
+ * larger.  Calls that take this path are ordered through one event per
+ * device, so calls on different streams or host threads never use the array
+ * at the same time (they may serialize on the GPU); under stream capture the
+ * ordering becomes external event nodes of the graph.  The first such call on
+ * a device looks up the array's address and creates the event: make it
+ * before any stream capture (q4_step_create does this itself).  When the
  * K dimension is split across thread blocks, y is zeroed on the stream and
  * the partial sums are added into it atomically, so the summation order (and
  * the last bits of y) may vary between runs.
@@ -184,15 +191,17 @@ q4_status q4_gemm(const uint8_t* codes, const uint16_t* scales,
  * q4_gemm_noalloc -- q4_gemm for callers that may not allocate device memory.
  * The paper has no counterpart; this entry point exists for deployment.
  *
- * q4_gemm's tensor-core path (M > 24) takes 2 * M * K bytes of scratch from
- * a memory pool (see Ownership).  Some callers cannot let a library do that: engines that
+ * Some callers cannot let a library allocate device memory: engines that
  * reserve all device memory at start-up for a fixed arena and a KV cache
- * leave no headroom for a pool that grows later, and hosts that account for
- * every byte themselves forbid hidden allocations.  This call computes the
- * same y with the same kernels, but keeps the binary16 copy of x in one
- * static device array of Q4_NOALLOC_SCRATCH_BYTES (8 MiB), which every GPU
- * that loads the library holds until the process exits.  It calls no
- * cudaMalloc, cudaFree or pool routine.
+ * leave no headroom for allocations that come later, and hosts that account
+ * for every byte themselves forbid hidden allocations.  q4_gemm allocates
+ * nothing either, but it orders the users of its fixed array through an
+ * event it creates, and it splits large inputs into chunks.  This call runs
+ * the same kernels without that event or chunking: it keeps the binary16
+ * copy of x in its own static device array of Q4_NOALLOC_SCRATCH_BYTES
+ * (8 MiB), which every GPU that loads the library holds until the process
+ * exits.  Its y agrees with q4_gemm's within the tolerance of q4_gemm.  It
+ * calls no cudaMalloc, cudaFree, pool or event routine.
  *
  * Limits and hazards:
  *   - M > 16 needs 2 * M * K <= Q4_NOALLOC_SCRATCH_BYTES (e.g. M = 512 at

@@ -440,6 +440,70 @@ def test_llama2_70b_prefill(linear, M):
     assert ok, f"{linear} M={M}: worst err/bound = {worst:.3g}"
 
 
+def test_tensor_core_path_allocates_nothing():
+    """q4_gemm at M > 24 keeps the binary16 copy of x in the library's fixed
+    array: after a warm-up call has loaded the kernels, a call whose copy of x
+    takes 29 MB (M = 512, K = 28672) leaves the device's free memory
+    unchanged, and its y matches the oracle on the strip rows."""
+    K, N, M = 28672, 256, 512
+    codes, scales = random_packed(41, N, K)
+    c, s, cb = dev_u8(codes), dev_u16(scales), dev_u16(NF4)
+    x = synth.activations(42, M, K)
+    xd = dev_u16(x)
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    warm_x = torch.zeros((32, K), dtype=torch.int16, device="cuda")
+    warm_y = torch.empty((32, N), dtype=torch.float32, device="cuda")
+    q4.q4_gemm(c, s, cb, warm_x, warm_y)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    q4.q4_gemm(c, s, cb, xd, y)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free0 - free1 < 2 * M * K // 2, (free0, free1)
+    rows = strip_rows(N, 3, n_random=64)
+    y_ref, a = oracle_matmul_parallel(codes, scales, NF4, x, rows=rows)
+    ok, worst = within_tolerance(y.cpu().numpy()[:, rows], y_ref, a)
+    assert ok, f"worst err/bound = {worst:.3g}"
+
+
+def test_tensor_core_path_chunks_large_inputs():
+    """An input whose binary16 copy (34 MB: M = 600, K = 28672) is larger than
+    the 32 MiB array runs in two chunks of tokens; every token row matches the
+    oracle on the strip rows."""
+    K, N, M = 28672, 130, 600
+    codes, scales = random_packed(43, N, K)
+    x = synth.activations(44, M, K)
+    y = run_matmul(codes, scales, NF4, x)
+    rows = strip_rows(N, 5, n_random=16)
+    y_ref, a = oracle_matmul_parallel(codes, scales, NF4, x, rows=rows)
+    ok, worst = within_tolerance(y[:, rows], y_ref, a)
+    assert ok, f"worst err/bound = {worst:.3g}"
+
+
+def test_tensor_core_path_two_streams():
+    """Tensor-core calls on two streams at once share the library's array
+    only one at a time: both results match the oracle."""
+    cb = dev_u16(NF4)
+    cases = []
+    for i, (M, N, K) in enumerate(((256, 384, 8192), (300, 257, 4160))):
+        codes, scales = random_packed(50 + i, N, K)
+        x = synth.activations(60 + i, M, K)
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        cases.append((codes, scales, x, dev_u8(codes), dev_u16(scales), dev_u16(x), y))
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    torch.cuda.synchronize()
+    for _ in range(3):
+        for (codes, scales, x, c, s, xd, y), st in zip(cases, streams):
+            with torch.cuda.stream(st):
+                q4.q4_gemm(c, s, cb, xd, y)
+    torch.cuda.synchronize()
+    for codes, scales, x, c, s, xd, y in cases:
+        rows = strip_rows(codes.shape[0], 7, n_random=32)
+        y_ref, a = oracle_matmul_parallel(codes, scales, NF4, x, rows=rows)
+        ok, worst = within_tolerance(y.cpu().numpy()[:, rows], y_ref, a)
+        assert ok, f"worst err/bound = {worst:.3g}"
+
+
 def test_ring_streams_host_weights():
     """CopyRing: packed weights in pinned host memory give the y of the
     resident path (bit for bit at M = 1) and stay within the tolerance of the

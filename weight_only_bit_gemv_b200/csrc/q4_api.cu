@@ -356,6 +356,13 @@ q4_status q4_step_create(const q4_linear* linears, int64_t n, q4_step** step) {
     DeviceInfo dev;
     q4_status st = gate(&dev);
     if (st != Q4_OK) return st;
+    for (int64_t i = 0; i < n; ++i)
+        if (linears[i].M > 16 && linears[i].N > 0) {
+            // the tensor-core path's fixed x array and event, set up outside the capture
+            const cudaError_t e = prepare_prefill(dev);
+            if (e != cudaSuccess) return cuda_fail(e);
+            break;
+        }
     q4_step* r = new q4_step();
     r->device = dev.device;
     cudaError_t e = cudaStreamCreateWithFlags(&r->capture, cudaStreamNonBlocking);

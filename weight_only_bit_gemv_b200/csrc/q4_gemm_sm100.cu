@@ -508,30 +508,49 @@ cudaError_t launch_prefill_tc(const uint8_t* codes, const uint16_t* scales, cons
     return cudaGetLastError();
 }
 
-// Stream-ordered scratch for the binary16 copy of x: one pool per device that
-// keeps what it has mapped (release threshold: never), so steady-state calls
-// neither map memory nor synchronize.
-static cudaError_t scratch_pool(int device, cudaMemPool_t* out) {
-    static std::mutex mu;
-    static cudaMemPool_t pools[64] = {};
+// ---------------------------------------------------------------------------
+// q4_gemm's binary16 copy of x: a fixed device array and an ordering event
+// ---------------------------------------------------------------------------
+// The tensor-core kernel streams x as binary16 by TMA; q4_gemm converts x into
+// this array first.  The array is part of the library's image (every GPU that
+// loads the library holds it until the process exits), so q4_gemm allocates
+// nothing at run time.  One event per device orders the calls that use it:
+// each call makes its stream wait for the previous user's kernels (on
+// whatever stream) before it writes the array, and records the event after
+// its own GEMM, so calls on different streams never use the array at the same
+// time.  Under stream capture the wait and the record become external event
+// nodes of the graph, so graph replays are ordered the same way.  Inputs
+// whose binary16 copy is larger than the array run in chunks of tokens.
+// (Converting x inside the kernel instead measured 1.5-1.8x slower at 256 and
+// 512 tokens on B200: the conversion doubles the shared-memory traffic of the
+// x tiles, and that traffic already bounds the 256-token tile.)
+static __device__ __align__(256) uint16_t g_gemm_x[kGemmXBytes / sizeof(uint16_t)];
+
+namespace {
+struct GemmXScratch {
+    uint16_t* addr = nullptr;
+    cudaEvent_t last = nullptr;  // recorded after the latest GEMM that read the array
+};
+std::mutex g_gemm_x_mu;  // also makes each call's wait / launch / record sequence atomic
+GemmXScratch g_gemm_x_dev[64];
+
+// The array's device address and the device's event, set up on first use
+// with `device` current.
+cudaError_t gemm_x_scratch(int device, GemmXScratch** out) {
     if (device < 0 || device >= 64) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!pools[device]) {
-        cudaMemPoolProps props{};
-        props.allocType = cudaMemAllocationTypePinned;
-        props.location.type = cudaMemLocationTypeDevice;
-        props.location.id = device;
-        cudaMemPool_t pool;
-        cudaError_t e = cudaMemPoolCreate(&pool, &props);
+    GemmXScratch& sc = g_gemm_x_dev[device];
+    if (!sc.addr) {
+        void* a = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&a, g_gemm_x);
         if (e != cudaSuccess) return e;
-        uint64_t keep = ~0ull;
-        e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        e = cudaEventCreateWithFlags(&sc.last, cudaEventDisableTiming);
         if (e != cudaSuccess) return e;
-        pools[device] = pool;
+        sc.addr = static_cast<uint16_t*>(a);
     }
-    *out = pools[device];
+    *out = &sc;
     return cudaSuccess;
 }
+}  // namespace
 
 cudaError_t take_gemm_tc_error(unsigned int* out) {
     unsigned int zero = 0;
@@ -540,18 +559,38 @@ cudaError_t take_gemm_tc_error(unsigned int* out) {
     return e;
 }
 
+cudaError_t prepare_prefill(const DeviceInfo& dev) {
+    std::lock_guard<std::mutex> lock(g_gemm_x_mu);
+    GemmXScratch* sc = nullptr;
+    return gemm_x_scratch(dev.device, &sc);
+}
+
 cudaError_t launch_prefill(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
                            cudaStream_t s, const DeviceInfo& dev) {
-    cudaMemPool_t pool;
-    cudaError_t e = scratch_pool(dev.device, &pool);
+    std::lock_guard<std::mutex> lock(g_gemm_x_mu);
+    GemmXScratch* sc = nullptr;
+    cudaError_t e = gemm_x_scratch(dev.device, &sc);
     if (e != cudaSuccess) return e;
-    void* xh = nullptr;
-    e = cudaMallocFromPoolAsync(&xh, static_cast<size_t>(M) * K * sizeof(uint16_t), pool, s);
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(s, &cs);
     if (e != cudaSuccess) return e;
-    e = launch_prefill_tc(codes, scales, cb, x, static_cast<uint16_t*>(xh), y, M, N, K, s, dev);
-    const cudaError_t f = cudaFreeAsync(xh, s);
-    return e != cudaSuccess ? e : f;
+    const bool capturing = cs != cudaStreamCaptureStatusNone;
+    // tokens per chunk: as many as the array holds, balanced over the chunks
+    const int64_t cap = static_cast<int64_t>(kGemmXBytes / (2 * static_cast<size_t>(K)));
+    const int64_t chunks = (M + cap - 1) / cap;
+    const int64_t per = (M + chunks - 1) / chunks;
+    for (int64_t m0 = 0; m0 < M; m0 += per) {
+        const int64_t mc = M - m0 < per ? M - m0 : per;
+        e = cudaStreamWaitEvent(s, sc->last, capturing ? cudaEventWaitExternal : cudaEventWaitDefault);
+        if (e != cudaSuccess) return e;
+        e = launch_prefill_tc(codes, scales, cb, x + m0 * K, sc->addr, y + m0 * N, mc, N, K, s, dev);
+        if (e != cudaSuccess) return e;
+        e = capturing ? cudaEventRecordWithFlags(sc->last, s, cudaEventRecordExternal)
+                      : cudaEventRecord(sc->last, s);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 // ---------------------------------------------------------------------------

@@ -58,10 +58,19 @@ cudaError_t launch_gemm_small(const uint8_t* codes, const uint16_t* scales, cons
                               const uint16_t* x, float* y, int M, int64_t N, int64_t K,
                               cudaStream_t s, const DeviceInfo& dev);
 // M > 24 (and M = 17..24 when launch_gemm_small declines the shape):
-// tcgen05 tensor-core GEMM with TMEM accumulators.
+// tcgen05 tensor-core GEMM with TMEM accumulators; x is converted to
+// binary16 into a fixed device array whose users are ordered by one event
+// per device.
+// prepare_prefill sets up that array's address and event on `dev` (current):
+// call it before a stream capture that may record the first such GEMM.
+cudaError_t prepare_prefill(const DeviceInfo& dev);
 cudaError_t launch_prefill(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
                            const uint16_t* x, float* y, int64_t M, int64_t N, int64_t K,
                            cudaStream_t s, const DeviceInfo& dev);
+
+// Size of q4_gemm's fixed device array for the binary16 copy of x (32 MiB
+// per GPU); larger inputs run in chunks of tokens.
+constexpr size_t kGemmXBytes = 32u << 20;
 
 // launch_prefill with the x scratch in a fixed device array (q4_gemm_noalloc); the
 // caller has checked 2 * M * K <= Q4_NOALLOC_SCRATCH_BYTES.
