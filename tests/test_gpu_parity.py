@@ -275,6 +275,23 @@ def test_integer_codebook_exact(M):
         assert np.array_equal(run_matmul(codes, scales, cb, x, "gemv"), y_ref)
 
 
+@pytest.mark.parametrize("N", [1, 15, 17, 33, 300, 4099])
+def test_gemv_rows_of_2kb(N):
+    """One token with K = 4096 (codes loaded straight into registers): ragged
+    N (a partial last tile, fewer rows than a tile, one row) against the
+    oracle, and the integer codebook exactly."""
+    K = 4096
+    codes, scales = random_packed(800 + N, N, K)
+    x = synth.activations(801 + N, 1, K)
+    assert_close(run_matmul(codes, scales, NF4, x, "gemv"), codes, scales, NF4, x, label=f"N={N}")
+    rng = np.random.default_rng(N)
+    cb = synth.integer_codebook()
+    sc = np.asarray(2.0 ** rng.integers(0, 3, size=(N, K // GROUP)), np.float16).view(np.uint16)
+    xi = synth.f32_to_bf16_bits(rng.integers(-4, 5, size=(1, K)).astype(np.float32))
+    y_ref, _ = oracle.matmul(codes, sc, cb, xi)
+    assert np.array_equal(run_matmul(codes, sc, cb, xi, "gemv"), y_ref)
+
+
 @pytest.mark.parametrize("M,N,K", [(40, 300, 64), (300, 130, 640), (257, 64, 1088),
                                    (20, 1, 256), (512, 129, 192)])
 def test_integer_codebook_exact_prefill_shapes(M, N, K):
