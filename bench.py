@@ -58,11 +58,12 @@ def peaks():
 # (4096 -> 22016) from an ncu capture, with the SHA-1 of the kernel source it
 # was taken on; when the source changes the figure no longer applies and the
 # bench reports null.
-GEMV_TRAFFIC = {"bytes": 47952128 + 7680,
-                "source_sha1": "1da9f429fe162a2b3c7c184dc784cef12b76512d",
-                "capture": "ncu --set full --clock-control none -k regex:gemv_m1 -s 2 -c 1 "
-                           "python -m weight_only_bit_gemv_b200.profile_case --M 1 --iters 5 "
-                           "--copies 2 --workload llama2_7b_layer --linear gate_up"}
+GEMV_TRAFFIC = {"bytes": 47953152 + 0,
+                "source_sha1": "38ec304025d8d3e5829d96ca86d3f7fe37bbf31d",
+                "capture": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
+                           "--clock-control none -k regex:gemv_m1 -s 2 -c 1 python -m "
+                           "weight_only_bit_gemv_b200.profile_case --workload llama2_7b_layer "
+                           "--linear gate_up --M 1 --iters 5 --copies 2"}
 
 
 def gemv_traffic():
@@ -297,26 +298,30 @@ def run_ours(args, world, rank, local):
     per_ms = [statistics.mean(p) for p in per]
     dom = max(range(len(lins)), key=lambda j: algo_bytes(1, lins[j]["lin"].N, lins[j]["lin"].K))
     dom_bytes = algo_bytes(1, lins[dom]["lin"].N, lins[dom]["lin"].K)
-    # The dominant kernel timed on its own: one graph of COPIES back-to-back
-    # launches over the rotating weight copies (events around the graph; an
-    # event between launches would also time the launch gap it creates).
-    Ld = lins[dom]
-    g_dom = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_dom, stream=stream):
-        for c in range(COPIES):
-            q4.q4_gemv(Ld["copies"][c][0], Ld["copies"][c][1], cb, Ld["x"], Ld["y"])
-    reps_dom = max(4, min(K, 200))
-    d0 = torch.cuda.Event(enable_timing=True)
-    d1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            g_dom.replay()
-        d0.record()
-        for _ in range(reps_dom):
-            g_dom.replay()
-        d1.record()
-    d1.synchronize()
-    dom_ms = d0.elapsed_time(d1) / (reps_dom * COPIES)
+    # Each linear timed on its own: one graph of COPIES back-to-back launches
+    # over the rotating weight copies, events around the graph (an event
+    # between launches would also time the launch gap it creates).  The
+    # dominant one is the roofline kernel.
+    def alone_ms(L):
+        g_one = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_one, stream=stream):
+            for c in range(COPIES):
+                q4.q4_gemv(L["copies"][c][0], L["copies"][c][1], cb, L["x"], L["y"])
+        reps_one = max(4, min(K, 200))
+        d0 = torch.cuda.Event(enable_timing=True)
+        d1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g_one.replay()
+            d0.record()
+            for _ in range(reps_one):
+                g_one.replay()
+            d1.record()
+        d1.synchronize()
+        return d0.elapsed_time(d1) / (reps_one * COPIES)
+
+    alone = [alone_ms(L) for L in lins]
+    dom_ms = alone[dom]
     dom_gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
 
     # ---- end to end through the Python API with host buffers -----------------
@@ -397,10 +402,10 @@ def run_ours(args, world, rank, local):
         cpu = cpu_baseline(lins, cb, args.cpu_seconds)
         cpu["coverage"] = cpu_coverage()
 
-    # per-linear launch time as a fixed cost plus bytes over a streaming rate
-    # (least squares over the step's four linears)
+    # per-linear launch time, each linear back to back on its own, as a fixed
+    # cost plus bytes over a streaming rate (least squares over the four)
     xb = np.array([algo_bytes(1, L["lin"].N, L["lin"].K) for L in lins], dtype=np.float64)
-    tb = np.array([statistics.median(p) * 1e3 for p in per], dtype=np.float64)  # us
+    tb = np.array([a * 1e3 for a in alone], dtype=np.float64)  # us
     slope, fixed = np.polyfit(xb, tb, 1)
     fit = f"{fixed:.2f} us fixed + bytes at {1e-3 / slope:.0f} GB/s" if slope > 0 else "n/a"
 
@@ -426,10 +431,12 @@ def run_ours(args, world, rank, local):
                   f"({COPIES * sum(L['copies'][0][0].numel() + 2 * L['copies'][0][1].numel() for L in lins) / 1e6:.0f} MB)",
             "launch": "CUDA graphs of the step's four launches",
             "hbm_frac_of_" + peak_src: round(value / world / hbm_peak, 4),
-            "per_linear_us": {L["lin"].name: round(per_ms[j] * 1e3, 3) for j, L in enumerate(lins)},
+            "per_linear_us_in_step_events": {L["lin"].name: round(per_ms[j] * 1e3, 3) for j, L in enumerate(lins)},
             "per_linear_us_p10_p50_p90": {L["lin"].name: pcts(per[j]) for j, L in enumerate(lins)},
             "decode_tok_s_equiv_32_layers": round(1e3 / (ms_step * 32), 1),
-            "per_linear_us_p10_p50_p90_str": "; ".join(
+            "per_linear_us_back_to_back": "; ".join(
+                f"{L['lin'].name} {alone[j] * 1e3:.2f}" for j, L in enumerate(lins)),
+            "per_linear_us_in_step_p10_p50_p90": "; ".join(
                 f"{L['lin'].name} " + "/".join(f"{v:.2f}" for v in pcts(per[j])) for j, L in enumerate(lins)),
             "per_linear_fit": fit,
         },
