@@ -364,9 +364,27 @@ struct G2 {
     int NS;     // ring stages
     int PT;     // tiles per pass of the partial slots
     int units;  // units of a row (ceil(R / 128))
+    uint32_t slot_off;  // per-warp row partials (after the table when there is one)
     uint32_t bar_off, x_off, zero_off, ring_off, stage_bytes, scale_off;
     SelMul k;
 };
+
+// Dynamic shared memory starts at this shared-window address on sm_100 (the
+// launcher checks the device's reservation), so a table at its start is read
+// with the address in the load's immediate.
+constexpr uint32_t kR2Base = 1024;
+constexpr uint32_t kR2LutBytes = 65536;  // 256 byte values x 32 lanes x 8 bytes
+
+// Table entry of code byte `byte` of w for this lane: the binary16 pairs
+// (cb[c0], cb[c1]) and (cb[c2], cb[c3]) of its four codes.
+template <int kByte>
+__device__ __forceinline__ uint2 lut2(uint32_t w, uint32_t lane8) {
+    uint2 v;
+    asm("ld.shared.v2.b32 {%0, %1}, [%2 + %3];"
+        : "=r"(v.x), "=r"(v.y)
+        : "r"(__byte_perm(w, lane8, 0x5504 | (kByte << 4))), "n"(kR2Base));
+    return v;
+}
 
 __device__ __forceinline__ uint4 lds128_v(uint32_t addr) {
     uint4 v;
@@ -421,7 +439,12 @@ __device__ __forceinline__ void copy_scales(uint32_t dst, const uint16_t* src) {
 
 // kWhole: a tile is one stage (rows of at most 2 KB); kSW: bytes per scale
 // copy (16, 8, 4 with cp.async; 2 = plain loads, for an odd group count).
-template <bool kWhole, int kSW>
+// kLut: word quarters q = 0, 1 of every group are decoded through a per-lane
+// byte -> four binary16 values table in shared memory (one LDS.64 and one PRMT
+// per four weights) instead of by PRMT from the codebook registers (about 2.4
+// ALU instructions per weight), which moves half of the decode from the ALU
+// pipe to the shared-memory pipe.
+template <bool kWhole, int kSW, bool kLut>
 __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -429,6 +452,11 @@ __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const uint32_t base = smem_u32(smem);
+    if (kLut && base != kR2Base) {
+        // the table's immediate addressing does not hold: report, write nothing
+        if (tid == 0) atomicOr(&g_gemv2_error, 0x1u);
+        return;
+    }
     const uint32_t bars = base + p.bar_off;
     const int NS = p.NS;
     const int r0 = static_cast<int>(static_cast<int64_t>(p.N) * blockIdx.x / gridDim.x);
@@ -527,7 +555,7 @@ __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
     }
 
     // ------------------------------- consumers ------------------------------
-    float* acc_s = reinterpret_cast<float*>(smem);  // [PT tiles][kR2CW warps][16 rows]
+    float* acc_s = reinterpret_cast<float*>(smem + p.slot_off);  // [PT tiles][kR2CW warps][16 rows]
     const int upk = kWhole ? p.units : p.KC / kR2Unit;
     const uint32_t off1 = 32 * tq + 16 * (g & 1), off2 = 32 * tq + 16 * (1 - (g & 1));
     const bool swap = (g & 1) != 0;
@@ -546,24 +574,46 @@ __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
         cbh |= (hv >> 8) << (8 * e);
     }
     {
-        // x of every unit as binary16 in MMA order: MMA m = 8 q + 2 i + h of
-        // group 8 u + a holds (x[16 q + 8 h + i], x[16 q + 8 h + 4 + i]) of the
-        // group, at x_off + 1024 u + 128 (m / 4) + 16 a + 4 (m % 4); zeros
-        // past the last group
-        const int items = p.units * 8 * 8;  // (unit, a, q, h)
+        // x of every unit as binary16 in MMA order, at x_off + 1024 u +
+        // 128 (m / 4) + 16 a + 4 (m % 4) for MMA m = 8 q + 2 i + h of group
+        // 8 u + a; zeros past the last group.  A quarter decoded by PRMT
+        // takes code i of bytes 2 h, 2 h + 1 of its word: (x[16 q + 8 h + i],
+        // x[16 q + 8 h + 4 + i]).  A quarter decoded by the table takes codes
+        // 2 h, 2 h + 1 of byte i: (x[16 q + 4 i + 2 h], x[16 q + 4 i + 2 h + 1]).
+        const int items = p.units * 8 * 4;  // (unit, a, q)
         for (int it = tid; it < items; it += kR2CW * 32) {
-            const int h = it & 1, q = (it >> 1) & 3, a = (it >> 3) & 7, u = it >> 6;
+            const int q = it & 3, a = (it >> 2) & 7, u = it >> 5;
             const int grp = 8 * u + a;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (grp < p.G)
-                v = __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(grp) * kGroup + 16 * q + 8 * h));
-            const uint32_t e[8] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16,
-                                   v.z & 0xFFFFu, v.z >> 16, v.w & 0xFFFFu, v.w >> 16};
+            uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+            if (grp < p.G) {
+                const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(grp) * kGroup + 16 * q);
+                v0 = __ldg(src);
+                v1 = __ldg(src + 1);
+            }
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            const bool by_table = kLut && q < 2;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int m = 8 * q + 2 * i + h;
-                *reinterpret_cast<uint32_t*>(smem + p.x_off + 1024 * u + 128 * (m >> 2) + 16 * a + 4 * (m & 3)) =
-                    bf16pair_to_f16x2(e[i], e[4 + i]);
+            for (int mm = 0; mm < 8; ++mm) {
+                const int i = mm >> 1, h = mm & 1, m = 8 * q + mm;
+                uint32_t pair;
+                if (by_table) {
+                    pair = bf16pair_to_f16x2(w[2 * i + h] & 0xFFFFu, w[2 * i + h] >> 16);
+                } else {
+                    const int e0 = 8 * h + i, e1 = 8 * h + 4 + i;
+                    pair = bf16pair_to_f16x2((w[e0 >> 1] >> (16 * (e0 & 1))) & 0xFFFFu,
+                                             (w[e1 >> 1] >> (16 * (e1 & 1))) & 0xFFFFu);
+                }
+                *reinterpret_cast<uint32_t*>(smem + p.x_off + 1024 * u + 128 * (m >> 2) + 16 * a + 4 * (m & 3)) = pair;
+            }
+        }
+        if (kLut) {
+            // entry of byte value v for lane l at 256 v + 8 l: (cb[c0], cb[c1]), (cb[c2], cb[c3])
+            for (int it = tid; it < 256 * 16; it += kR2CW * 32) {
+                const int v = it >> 4;
+                const uint32_t c0 = __ldg(p.cb + (v & 3)), c1 = __ldg(p.cb + ((v >> 2) & 3));
+                const uint32_t c2 = __ldg(p.cb + ((v >> 4) & 3)), c3 = __ldg(p.cb + (v >> 6));
+                const uint32_t e01 = c0 | (c1 << 16), e23 = c2 | (c3 << 16);
+                *reinterpret_cast<uint4*>(smem + 256 * v + 16 * (it & 15)) = make_uint4(e01, e23, e01, e23);
             }
         }
         for (int it = tid; it < 1024 / 16; it += kR2CW * 32)
@@ -603,6 +653,36 @@ __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
                         const uint32_t xb1[8] = {xw0.x, xw0.y, xw0.z, xw0.w, xw1.x, xw1.y, xw1.z, xw1.w};
                         const uint32_t wlg = word4(lo_g, q), whg = word4(hi_g, q);
                         const uint32_t wlh = word4(lo_h, q), whh = word4(hi_h, q);
+                        if (kLut && q < 2) {
+                            const uint32_t lane8 = static_cast<uint32_t>(lane) * 8u;
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                uint2 tlg, tlh, thg, thh;
+                                switch (i) {
+                                    case 0:
+                                        tlg = lut2<0>(wlg, lane8); tlh = lut2<0>(wlh, lane8);
+                                        thg = lut2<0>(whg, lane8); thh = lut2<0>(whh, lane8);
+                                        break;
+                                    case 1:
+                                        tlg = lut2<1>(wlg, lane8); tlh = lut2<1>(wlh, lane8);
+                                        thg = lut2<1>(whg, lane8); thh = lut2<1>(whh, lane8);
+                                        break;
+                                    case 2:
+                                        tlg = lut2<2>(wlg, lane8); tlh = lut2<2>(wlh, lane8);
+                                        thg = lut2<2>(whg, lane8); thh = lut2<2>(whh, lane8);
+                                        break;
+                                    default:
+                                        tlg = lut2<3>(wlg, lane8); tlh = lut2<3>(wlh, lane8);
+                                        thg = lut2<3>(whg, lane8); thh = lut2<3>(whh, lane8);
+                                        break;
+                                }
+                                uint32_t a[4] = {tlg.x, tlh.x, thg.x, thh.x};
+                                mma_16816(d0, a, xb0[2 * i], xb1[2 * i], d0);
+                                uint32_t a2[4] = {tlg.y, tlh.y, thg.y, thh.y};
+                                mma_16816(d1, a2, xb0[2 * i + 1], xb1[2 * i + 1], d1);
+                            }
+                            continue;
+                        }
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             uint32_t slg0, slg1, shg0, shg1, slh0, slh1, shh0, shh1;
@@ -688,9 +768,9 @@ __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
     }
 }
 
-template <bool kWhole, int kSW>
+template <bool kWhole, int kSW, bool kLut>
 cudaError_t launch_ring2(const G2& p, int grid, int smem, int slot, cudaStream_t s, const DeviceInfo& dev) {
-    auto kern = gemv2_ring_kernel<kWhole, kSW>;
+    auto kern = gemv2_ring_kernel<kWhole, kSW, kLut>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem, slot, dev.device);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -738,14 +818,24 @@ cudaError_t launch_gemv2_ring(const uint8_t* codes, const uint16_t* scales, cons
     p.scale_off = code_bytes;
     p.stage_bytes = code_bytes + ((static_cast<uint32_t>(16 * p.GS * 2) + 127u) & ~127u);
     const uint32_t x_bytes = static_cast<uint32_t>(p.units) * 1024u;
+    uint32_t head = 0;  // the table, when there is one, ahead of everything else
     auto layout = [&](int pt) {
         p.PT = pt;
-        p.bar_off = static_cast<uint32_t>(pt) * kR2TileSlotBytes;
+        p.slot_off = head;
+        p.bar_off = head + static_cast<uint32_t>(pt) * kR2TileSlotBytes;
         p.zero_off = p.bar_off + 128u;
         p.x_off = p.zero_off + 1024u;
         p.ring_off = (p.x_off + x_bytes + 127u) & ~127u;
         return dev.smem_optin - static_cast<int>(p.ring_off);
     };
+    // the table needs the dynamic shared-memory base at kR2Base and room for
+    // at least three ring stages beside it
+    bool lut = dev.smem_reserved == static_cast<int>(kR2Base);
+    if (lut) {
+        head = kR2LutBytes;
+        lut = layout(kR2MinPassTiles) / static_cast<int>(p.stage_bytes) >= 3;
+    }
+    if (!lut) head = 0;
     int ns = layout(kR2MinPassTiles) / static_cast<int>(p.stage_bytes);
     if (ns > kR2MaxStages) ns = kR2MaxStages;
     if (ns < 2) return cudaErrorNotSupported;
@@ -761,20 +851,27 @@ cudaError_t launch_gemv2_ring(const uint8_t* codes, const uint16_t* scales, cons
     const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
     // widest scale copy that every source and destination offset allows
     const int gcd_groups = p.G % 8 == 0 && p.GS % 8 == 0 ? 8 : (p.G % 4 == 0 && p.GS % 4 == 0 ? 4 : (p.G % 2 == 0 && p.GS % 2 == 0 ? 2 : 1));
+    // slots 51..58 without the table, 59..66 with it
+    const int slot = 51 + (whole ? 0 : 4) + (gcd_groups == 8 ? 0 : gcd_groups == 4 ? 1 : gcd_groups == 2 ? 2 : 3) +
+                     (lut ? 8 : 0);
+#define Q4_RING2(W, SW)                                                                  \
+    return lut ? launch_ring2<W, SW, true>(p, grid, smem, slot, s, dev)                  \
+               : launch_ring2<W, SW, false>(p, grid, smem, slot, s, dev)
     if (whole) {
         switch (gcd_groups) {
-            case 8: return launch_ring2<true, 16>(p, grid, smem, 51, s, dev);
-            case 4: return launch_ring2<true, 8>(p, grid, smem, 52, s, dev);
-            case 2: return launch_ring2<true, 4>(p, grid, smem, 53, s, dev);
-            default: return launch_ring2<true, 2>(p, grid, smem, 54, s, dev);
+            case 8: Q4_RING2(true, 16);
+            case 4: Q4_RING2(true, 8);
+            case 2: Q4_RING2(true, 4);
+            default: Q4_RING2(true, 2);
         }
     }
     switch (gcd_groups) {
-        case 8: return launch_ring2<false, 16>(p, grid, smem, 55, s, dev);
-        case 4: return launch_ring2<false, 8>(p, grid, smem, 56, s, dev);
-        case 2: return launch_ring2<false, 4>(p, grid, smem, 57, s, dev);
-        default: return launch_ring2<false, 2>(p, grid, smem, 58, s, dev);
+        case 8: Q4_RING2(false, 16);
+        case 4: Q4_RING2(false, 8);
+        case 2: Q4_RING2(false, 4);
+        default: Q4_RING2(false, 2);
     }
+#undef Q4_RING2
 }
 
 }  // namespace

@@ -9,7 +9,7 @@ namespace q4 {
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxSlots = 64;
+constexpr int kMaxSlots = 96;
 
 struct Cache {
     std::mutex mu;
