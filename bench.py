@@ -59,7 +59,7 @@ def peaks():
 # was taken on; when the source changes the figure no longer applies and the
 # bench reports null.
 GEMV_TRAFFIC = {"bytes": 47953152 + 0,
-                "source_sha1": "38ec304025d8d3e5829d96ca86d3f7fe37bbf31d",
+                "source_sha1": "dedcf912d557a0e31a9d3a1eb0f8526aac59428a",
                 "capture": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
                            "--clock-control none -k regex:gemv_m1 -s 2 -c 1 python -m "
                            "weight_only_bit_gemv_b200.profile_case --workload llama2_7b_layer "

@@ -370,6 +370,28 @@ q4_status q4_step_destroy(q4_step* step);
 q4_status q4_wait_selftest(uint32_t limit_us, int arrive, uint32_t* waited_us);
 
 /*
+ * Bounds-checked build.  Built with -DQ4_DEBUG (python -m
+ * weight_only_bit_gemv_b200.build --debug, which writes libq4_debug.so), every
+ * kernel checks the global index ranges it computes -- bulk-copy and load
+ * sources, scale copies, x reads, y writes -- against the buffers' extents
+ * before each access.  A range that falls outside sets a bit and the access
+ * is skipped (nothing traps; a skipped bulk copy leaves its mbarrier short and
+ * the waits behind it run out and report through q4_timeout_flags).  Not an
+ * operation of the method: a substitute for a memory checker.
+ *
+ * q4_bounds_flags -- synchronize the current device, store in *flags the bits
+ * set by failed checks since the last call and clear them: bit 0 the M <= 4
+ * decode kernel, 1 the M = 2..24 kernel, 2 the tensor-core GEMM, 3 the
+ * fallback small-M kernel, 4 pack / dequant / embedding rows, 5 the two-bit
+ * kernels.  Always 0 in a release build.  Returns Q4_ERR_NULL for a NULL
+ * flags, Q4_ERR_CUDA if a CUDA call fails.
+ *
+ * q4_bounds_checked -- 1 if this library was built with the checks, else 0.
+ */
+q4_status q4_bounds_flags(uint32_t* flags);
+int q4_bounds_checked(void);
+
+/*
  * q4_timeout_flags -- every wait inside the bulk-copy and tensor-core
  * kernels is bounded (about two seconds); a wait that runs out sets a bit in
  * a device word, the kernel drains what it has in flight, frees its tensor

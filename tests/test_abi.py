@@ -191,3 +191,44 @@ def test_wait_selftest_rejects(lib):
     assert lib.q4_wait_selftest(1000, 0, None) == NULL
     assert lib.q4_wait_selftest(0, 0, ctypes.byref(out)) == SHAPE
     assert lib.q4_wait_selftest(1000001, 1, ctypes.byref(out)) == SHAPE
+
+
+def test_bounds_flags_rejects_null(lib):
+    assert lib.q4_bounds_flags(None) == NULL
+
+
+def test_release_build_is_not_bounds_checked(lib):
+    if q4.debug_selected():
+        pytest.skip("Q4_LIBRARY=debug selects the bounds-checked build")
+    assert lib.q4_bounds_checked() == 0
+    assert q4.library_path().endswith("libq4.so")
+
+
+def test_library_selection_rejects_unknown_names(monkeypatch):
+    monkeypatch.setenv("Q4_LIBRARY", "fast")
+    with pytest.raises(RuntimeError):
+        q4.library_path()
+    monkeypatch.setenv("Q4_LIBRARY", "debug")
+    assert q4.library_path().endswith("libq4_debug.so")
+
+
+def test_debug_build_exports_the_same_and_says_so():
+    """libq4_debug.so (the -DQ4_DEBUG build) exports every declared function
+    and reports itself as bounds-checked; it is loaded in a child process,
+    since one process loads one of the two libraries."""
+    from weight_only_bit_gemv_b200 import build as b
+    b.build(debug=True)          # no-op when up to date
+    out = subprocess.run(["nm", "-D", "--defined-only", b.DEBUG_LIBRARY],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in q4.header_functions() if n not in exported]
+    assert not missing, missing
+    code = ("import ctypes, weight_only_bit_gemv_b200 as q4; l = q4.load(False); "
+            "print(q4.library_path(), l.q4_bounds_checked(), l.q4_bounds_flags(None))")
+    import os
+    import sys
+    env = dict(os.environ, Q4_LIBRARY="debug")
+    res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env,
+                         cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))), check=True)
+    path, checked, null_status = res.stdout.split()
+    assert path.endswith("libq4_debug.so") and checked == "1" and int(null_status) == NULL

@@ -5,6 +5,11 @@ the CUDA kernels of libq4.so, on the tensors' device, on the current torch
 stream.  PyTorch supplies device memory and streams.  There is no CPU path:
 if the library cannot be loaded, every call raises.
 
+Q4_LIBRARY=debug in the environment loads libq4_debug.so instead: the same
+kernels built with -DQ4_DEBUG, in which each global load and store checks its
+index range first and a failed check sets a bit of bounds_flags() and skips
+the access.  It is slower and meant for tests only.
+
 Tensor conventions (all contiguous, on one CUDA device):
   w        float32            [N, K]
   codebook float16 or uint16  [16]       (binary16 bits)
@@ -47,21 +52,32 @@ class Q4Linear(ctypes.Structure):
                 ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
 
 
+def debug_selected() -> bool:
+    """True when Q4_LIBRARY=debug selects the bounds-checked build."""
+    v = os.environ.get("Q4_LIBRARY", "").strip().lower()
+    if v not in ("", "release", "debug"):
+        raise RuntimeError(f"Q4_LIBRARY must be 'release' or 'debug', not {v!r}")
+    return v == "debug"
+
+
 def library_path() -> str:
-    return _build.LIBRARY
+    return _build.DEBUG_LIBRARY if debug_selected() else _build.LIBRARY
 
 
 def load(build_if_missing: bool = True) -> ctypes.CDLL:
-    """Load libq4.so (building it with nvcc first if it is missing or stale)."""
+    """Load libq4.so, or libq4_debug.so under Q4_LIBRARY=debug (building it
+    with nvcc first if it is missing or stale)."""
     global _lib
     if _lib is not None:
         return _lib
-    if build_if_missing and _build.stale():
-        _build.build()
-    if not os.path.exists(_build.LIBRARY):
-        raise RuntimeError(f"libq4.so not found at {_build.LIBRARY}; run "
-                           "python -m weight_only_bit_gemv_b200.build")
-    lib = ctypes.CDLL(_build.LIBRARY)
+    debug = debug_selected()
+    path = library_path()
+    if build_if_missing and _build.stale(path):
+        _build.build(debug=debug)
+    if not os.path.exists(path):
+        raise RuntimeError(f"{os.path.basename(path)} not found at {path}; run "
+                           "python -m weight_only_bit_gemv_b200.build" + (" --debug" if debug else ""))
+    lib = ctypes.CDLL(path)
     P, I64, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p
     lib.q4_pack.argtypes = [P, P, P, P, I64, I64, S]
     lib.q4_dequant.argtypes = [P, P, P, P, I64, I64, S]
@@ -97,6 +113,10 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.q4_step_destroy.restype = ctypes.c_int
     lib.q4_wait_selftest.argtypes = [ctypes.c_uint32, ctypes.c_int, ctypes.POINTER(ctypes.c_uint32)]
     lib.q4_wait_selftest.restype = ctypes.c_int
+    lib.q4_bounds_flags.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+    lib.q4_bounds_flags.restype = ctypes.c_int
+    lib.q4_bounds_checked.argtypes = []
+    lib.q4_bounds_checked.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -425,6 +445,19 @@ def timeout_flags() -> int:
     return int(out.value)
 
 
+def bounds_flags() -> int:
+    """Synchronize the current device; return and clear the bits of the
+    kernels' failed index checks (always 0 from the release build)."""
+    out = ctypes.c_uint32(0)
+    _check(load().q4_bounds_flags(ctypes.byref(out)), "q4_bounds_flags")
+    return int(out.value)
+
+
+def bounds_checked() -> bool:
+    """True when the loaded library is the bounds-checked build."""
+    return bool(load().q4_bounds_checked())
+
+
 def abi_version() -> int:
     return load().q4_abi_version()
 
@@ -474,3 +507,11 @@ def q4_step_destroy(step: Step) -> None:
 
 def q4_wait_selftest(limit_us: int, arrive: bool) -> int:
     return wait_selftest(limit_us, arrive)
+
+
+def q4_bounds_flags() -> int:
+    return bounds_flags()
+
+
+def q4_bounds_checked() -> bool:
+    return bounds_checked()

@@ -63,6 +63,10 @@ __global__ void __launch_bounds__(256) pack2_kernel(const float* __restrict__ w,
     for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
          idx += (int64_t)gridDim.x * blockDim.x) {
         const int64_t n = idx / G, g = idx - n * G;
+        if (!Q4_IN_BOUNDS(n * K + g * kGroup, kGroup, N * K) ||
+            !Q4_IN_BOUNDS(n * (K / 4) + g * (kGroup / 4), kGroup / 4, N * (K / 4)) ||
+            !Q4_IN_BOUNDS(n * G + g, 1, N * G))
+            continue;
         const float4* src = reinterpret_cast<const float4*>(w + n * K + g * kGroup);
         float v[kGroup];
 #pragma unroll
@@ -127,6 +131,9 @@ __global__ void __launch_bounds__(256) dequant2_kernel(const uint8_t* __restrict
          idx += (int64_t)gridDim.x * blockDim.x) {
         const int64_t n = idx / per_row, j = idx - n * per_row;
         const int64_t k0 = j * 16;
+        if (!Q4_IN_BOUNDS(n * (K / 4) + j * 4, 4, N * (K / 4)) || !Q4_IN_BOUNDS(n * G + k0 / kGroup, 1, N * G) ||
+            !Q4_IN_BOUNDS(n * K + k0, 16, N * K))
+            continue;
         const uint32_t word = __ldg(reinterpret_cast<const uint32_t*>(codes + n * (K / 4) + j * 4));
         const float s = half_bits_to_float2b(scales[n * G + k0 / kGroup]);
         float out[16];
@@ -171,11 +178,13 @@ __device__ __forceinline__ Q2Chunk load_chunk2(const uint8_t* __restrict__ codes
         const int64_t grp = 4 * ch + t;
         const int64_t ra = 16 * rt + g, rb = ra + 8;
         if (grp < G) {
-            if (ra < N) {
+            if (ra < N && Q4_IN_BOUNDS(ra * (K / 4) + grp * 16, 16, N * (K / 4)) &&
+                Q4_IN_BOUNDS(ra * G + grp, 1, N * G)) {
                 c.wa = __ldcs(reinterpret_cast<const uint4*>(codes + ra * (K / 4) + grp * 16));
                 c.sa = __ldg(reinterpret_cast<const unsigned short*>(scales + ra * G + grp));
             }
-            if (rb < N) {
+            if (rb < N && Q4_IN_BOUNDS(rb * (K / 4) + grp * 16, 16, N * (K / 4)) &&
+                Q4_IN_BOUNDS(rb * G + grp, 1, N * G)) {
                 c.wb = __ldcs(reinterpret_cast<const uint4*>(codes + rb * (K / 4) + grp * 16));
                 c.sb = __ldg(reinterpret_cast<const unsigned short*>(scales + rb * G + grp));
             }
@@ -201,7 +210,7 @@ __global__ void __launch_bounds__(kQ2Threads, 2)
         const int64_t grp = k / kGroup;
         const int r = static_cast<int>(k - grp * kGroup);
         const int q = r >> 4, j = (r >> 2) & 3, i = r & 3;
-        const __half h = __float2half_rn(bf16_bits_to_float(__ldg(x + k)));
+        const __half h = __float2half_rn(bf16_bits_to_float(Q4_IN_BOUNDS(k, 1, K) ? __ldg(x + k) : 0));
         *reinterpret_cast<__half*>(smem + grp * kQ2XGroupBytes + 8 * (4 * q + i) + 2 * j) = h;
     }
     __syncthreads();
@@ -232,8 +241,8 @@ __global__ void __launch_bounds__(kQ2Threads, 2)
         float vb = part_b + __shfl_xor_sync(0xFFFFFFFFu, part_b, 1);
         if (rt >= 0 && t == 0) {
             const int64_t ra = 16 * rt + g, rb = ra + 8;
-            if (ra < N) atomicAdd(y + ra, va);
-            if (rb < N) atomicAdd(y + rb, vb);
+            if (ra < N && Q4_IN_BOUNDS(ra, 1, N)) atomicAdd(y + ra, va);
+            if (rb < N && Q4_IN_BOUNDS(rb, 1, N)) atomicAdd(y + rb, vb);
         }
         part_a = 0.f;
         part_b = 0.f;
@@ -512,10 +521,12 @@ __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
             const int cbytes = kWhole ? p.R : min(p.KC, p.R - c * p.KC);
             if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(rows * cbytes));
             __syncwarp();
+            const int64_t code_extent = static_cast<int64_t>(p.N) * p.R;
             if (kWhole) {
-                if (lane == 0)
+                if (lane == 0 && Q4_IN_BOUNDS(static_cast<int64_t>(row0) * p.R, rows * p.R, code_extent))
                     bulk_load(dst, p.codes + static_cast<int64_t>(row0) * p.R, static_cast<uint32_t>(rows * p.R), full);
-            } else if (lane < rows) {
+            } else if (lane < rows &&
+                       Q4_IN_BOUNDS(static_cast<int64_t>(row0 + lane) * p.R + c * p.KC, cbytes, code_extent)) {
                 bulk_load(dst + lane * p.KC, p.codes + static_cast<int64_t>(row0 + lane) * p.R + c * p.KC,
                           static_cast<uint32_t>(cbytes), full);
             }
@@ -526,7 +537,9 @@ __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
             const uint32_t sdst = dst + p.scale_off;
             for (int j = lane; j < rows * per_row; j += 32) {
                 const int r = j / per_row, q = j - r * per_row;
-                copy_scales<kSW>(sdst + r * (p.GS * 2) + q * kSW,
+                if (Q4_IN_BOUNDS(static_cast<int64_t>(row0 + r) * p.G + g0 + q * (kSW / 2), kSW / 2,
+                                 static_cast<int64_t>(p.N) * p.G))
+                    copy_scales<kSW>(sdst + r * (p.GS * 2) + q * kSW,
                                  p.scales + static_cast<int64_t>(row0 + r) * p.G + g0 + q * (kSW / 2));
             }
             if (kSW > 2)
@@ -585,7 +598,7 @@ __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
             const int q = it & 3, a = (it >> 2) & 7, u = it >> 5;
             const int grp = 8 * u + a;
             uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
-            if (grp < p.G) {
+            if (grp < p.G && Q4_IN_BOUNDS(static_cast<int64_t>(grp) * kGroup + 16 * q, 16, p.K)) {
                 const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(grp) * kGroup + 16 * q);
                 v0 = __ldg(src);
                 v1 = __ldg(src + 1);
@@ -762,7 +775,7 @@ __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
             float sum = 0.f;
 #pragma unroll
             for (int w = 0; w < kR2CW; ++w) sum += q[16 * w];
-            p.y[r0 + r] = sum;
+            if (Q4_IN_BOUNDS(r0 + r, 1, p.N)) p.y[r0 + r] = sum;
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kR2CW * 32) : "memory");
     }
@@ -920,5 +933,7 @@ cudaError_t launch_gemv2(const uint8_t* codes, const uint16_t* scales, const uin
     gemv2_kernel<<<dev.sm_count * per_sm, kQ2Threads, smem, s>>>(codes, scales, cb, x, y, N, K);
     return cudaGetLastError();
 }
+
+Q4_DEFINE_TAKE_BOUNDS(gemv2)
 
 }  // namespace q4

@@ -417,6 +417,29 @@ q4_status q4_wait_selftest(uint32_t limit_us, int arrive, uint32_t* waited_us) {
     return e == cudaSuccess ? Q4_OK : cuda_fail(e);
 }
 
+q4_status q4_bounds_flags(uint32_t* flags) {
+    if (!flags) return Q4_ERR_NULL;
+    *flags = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    cudaError_t (*const take[6])(unsigned int*) = {take_bounds_gemv_m1, take_bounds_gemm_small,
+                                                   take_bounds_gemm_tc, take_bounds_gemv,
+                                                   take_bounds_pack, take_bounds_gemv2};
+    for (int i = 0; i < 6 && e == cudaSuccess; ++i) {
+        unsigned int v = 0;
+        e = take[i](&v);
+        if (v) *flags |= 1u << i;
+    }
+    return e == cudaSuccess ? Q4_OK : cuda_fail(e);
+}
+
+int q4_bounds_checked(void) {
+#ifdef Q4_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
 const char* q4_status_string(q4_status status) {
     switch (status) {
         case Q4_OK: return "Q4_OK";

@@ -201,14 +201,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int r = lane + 32 * jr;
                 const int row = strip * kR + r;
                 if (kAsyncScales) {
-                    const bool in = row < p.N;
+                    const bool in = row < p.N && Q4_IN_BOUNDS(static_cast<long long>(row) * p.G + g0, 4,
+                                                              static_cast<long long>(p.N) * p.G);
                     const uint16_t* src = in ? p.scales + static_cast<long long>(row) * p.G + g0 : p.scales;
                     cp_async_8(sdst + r * 8, src, in ? 8u : 0u);
                 } else {
 #pragma unroll
                     for (int q = 0; q < kWG; ++q) {
                         uint16_t v = 0;
-                        if (row < p.N && g0 + q < g_end)
+                        if (row < p.N && g0 + q < g_end &&
+                            Q4_IN_BOUNDS(static_cast<long long>(row) * p.G + g0 + q, 1,
+                                         static_cast<long long>(p.N) * p.G))
                             v = p.scales[static_cast<long long>(row) * p.G + g0 + q];
                         sts_u16(sdst + r * 8 + 2 * q, v);
                     }
@@ -368,7 +371,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int m = tt * p.BMT + c0 + e;
-                        if (n < p.N && m < p.M) {
+                        if (n < p.N && m < p.M &&
+                            Q4_IN_BOUNDS(static_cast<long long>(m) * p.N + n, 1,
+                                         static_cast<long long>(p.M) * p.N)) {
                             float* dst = p.y + static_cast<long long>(m) * p.N + n;
                             if (p.ksplit > 1)
                                 red_add_f32(dst, __uint_as_float(v[e]));
@@ -392,9 +397,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-__global__ void bf16_to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xh, int64_t n8) {
+// xh_elems: binary16 elements the destination array holds
+__global__ void bf16_to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xh, int64_t n8,
+                                   int64_t xh_elems) {
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        if (!Q4_IN_BOUNDS(8 * i, 8, xh_elems)) continue;
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + i);
         uint4 h;
         const uint32_t in[4] = {v.x, v.y, v.z, v.w};
@@ -416,8 +424,8 @@ __global__ void bf16_to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __r
 }  // namespace
 
 cudaError_t launch_prefill_tc(const uint8_t* codes, const uint16_t* scales, const uint16_t* cb,
-                              const uint16_t* x, uint16_t* xh, float* y, int64_t M, int64_t N,
-                              int64_t K, cudaStream_t s, const DeviceInfo& dev) {
+                              const uint16_t* x, uint16_t* xh, int64_t xh_elems, float* y, int64_t M,
+                              int64_t N, int64_t K, cudaStream_t s, const DeviceInfo& dev) {
     TcGemm p{};
     p.scales = scales;
     p.cb = cb;
@@ -468,7 +476,7 @@ cudaError_t launch_prefill_tc(const uint8_t* codes, const uint16_t* scales, cons
     const int64_t n8 = M * K / 8;
     int cgrid = static_cast<int>((n8 + 255) / 256);
     if (cgrid > dev.sm_count * 8) cgrid = dev.sm_count * 8;
-    bf16_to_f16_kernel<<<cgrid, 256, 0, s>>>(x, xh, n8);
+    bf16_to_f16_kernel<<<cgrid, 256, 0, s>>>(x, xh, n8, xh_elems);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -584,7 +592,8 @@ cudaError_t launch_prefill(const uint8_t* codes, const uint16_t* scales, const u
         const int64_t mc = M - m0 < per ? M - m0 : per;
         e = cudaStreamWaitEvent(s, sc->last, capturing ? cudaEventWaitExternal : cudaEventWaitDefault);
         if (e != cudaSuccess) return e;
-        e = launch_prefill_tc(codes, scales, cb, x + m0 * K, sc->addr, y + m0 * N, mc, N, K, s, dev);
+        e = launch_prefill_tc(codes, scales, cb, x + m0 * K, sc->addr, kGemmXBytes / 2, y + m0 * N, mc, N,
+                              K, s, dev);
         if (e != cudaSuccess) return e;
         e = capturing ? cudaEventRecordWithFlags(sc->last, s, cudaEventRecordExternal)
                       : cudaEventRecord(sc->last, s);
@@ -629,7 +638,9 @@ cudaError_t launch_prefill_noalloc(const uint8_t* codes, const uint16_t* scales,
     uint16_t* xh = nullptr;
     const cudaError_t e = noalloc_scratch(dev.device, &xh);
     if (e != cudaSuccess) return e;
-    return launch_prefill_tc(codes, scales, cb, x, xh, y, M, N, K, s, dev);
+    return launch_prefill_tc(codes, scales, cb, x, xh, Q4_NOALLOC_SCRATCH_BYTES / 2, y, M, N, K, s, dev);
 }
+
+Q4_DEFINE_TAKE_BOUNDS(gemm_tc)
 
 }  // namespace q4

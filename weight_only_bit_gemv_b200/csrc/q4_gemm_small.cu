@@ -123,10 +123,13 @@ __device__ __forceinline__ void load_stage_scales(const uint16_t* srow, int kb, 
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         if (kEvenG) {
-            out[i] = ldg_nc_u32(srow + min(g0 + 2 * i, G - 2));
+            const int g = min(g0 + 2 * i, G - 2);
+            out[i] = Q4_IN_BOUNDS(g, 2, G) ? ldg_nc_u32(srow + g) : 0u;
         } else {
-            out[i] = ldg_nc_u16(srow + min(g0 + 2 * i, G - 1)) |
-                     (ldg_nc_u16(srow + min(g0 + 2 * i + 1, G - 1)) << 16);
+            const int ga = min(g0 + 2 * i, G - 1), gb = min(g0 + 2 * i + 1, G - 1);
+            out[i] = Q4_IN_BOUNDS(ga, 1, G) && Q4_IN_BOUNDS(gb, 1, G)
+                         ? ldg_nc_u16(srow + ga) | (ldg_nc_u16(srow + gb) << 16)
+                         : 0u;
         }
     }
 }
@@ -229,7 +232,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int m = i / chunks, j = i - m * chunks;
                 const int k = k0 + 8 * j;
                 b[r] = make_uint4(0u, 0u, 0u, 0u);
-                if (i < total && k < p.K)
+                if (i < total && k < p.K &&
+                    Q4_IN_BOUNDS(static_cast<int64_t>(m) * p.K + k, 8, static_cast<int64_t>(p.M) * p.K))
                     b[r] = __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * p.K + k));
             }
 #pragma unroll
@@ -262,8 +266,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int nrb = rb_first, ns = 0;
     auto load_next = [&]() {
         if (nrb < p.NB) {
-            const int n1 = min(nrb * kRows + r1, p.N - 1), n2 = min(nrb * kRows + r1 + 8, p.N - 1);
+            int n1 = min(nrb * kRows + r1, p.N - 1), n2 = min(nrb * kRows + r1 + 8, p.N - 1);
             const int kb = k0 + ns * kStageK;
+            if (!Q4_IN_BOUNDS(n1, 1, p.N) || !Q4_IN_BOUNDS(n2, 1, p.N)) n1 = n2 = 0;
             load_stage_scales<kEvenG>(p.scales + static_cast<int64_t>(n1) * p.G, kb, p.G, nx_lo);
             load_stage_scales<kEvenG>(p.scales + static_cast<int64_t>(n2) * p.G, kb, p.G, nx_hi);
             if (++ns == nst) {
@@ -385,7 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int q = 0; q < 4; ++q) {
                 const int m = 8 * mb + 2 * tq + (q & 1);
                 const int n = rb * kRows + r1 + 8 * (q >> 1);
-                if (m < p.M && n < p.N) {
+                if (m < p.M && n < p.N &&
+                    Q4_IN_BOUNDS(static_cast<int64_t>(m) * p.N + n, 1, static_cast<int64_t>(p.M) * p.N)) {
                     float* dst = p.y + static_cast<int64_t>(m) * p.N + n;
                     if (p.KS > 1)
                         red_add_f32(dst, acc[mb][q]);
@@ -485,5 +491,7 @@ cudaError_t launch_gemm_small(const uint8_t* codes, const uint16_t* scales, cons
     return even ? launch_variant<4, true>(cmap, p, best_grid, smem, 46, s, dev)
                 : launch_variant<4, false>(cmap, p, best_grid, smem, 47, s, dev);
 }
+
+Q4_DEFINE_TAKE_BOUNDS(gemm_small)
 
 }  // namespace q4

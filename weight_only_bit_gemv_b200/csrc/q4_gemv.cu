@@ -83,8 +83,10 @@ __device__ void stage_x(const SmallM& p, uint32_t xs, int c0, int cn) {
     for (int u = threadIdx.x; u < total; u += kThreads) {
         const int m = u / units_per_row;
         const int r = u - m * units_per_row;
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(
-            p.x + static_cast<int64_t>(m) * p.K + static_cast<int64_t>(c0) * kGroup + r * 8));
+        const int64_t off = static_cast<int64_t>(m) * p.K + static_cast<int64_t>(c0) * kGroup + r * 8;
+        const uint4 v = Q4_IN_BOUNDS(off, 8, static_cast<int64_t>(p.M) * p.K)
+                            ? __ldg(reinterpret_cast<const uint4*>(p.x + off))
+                            : make_uint4(0u, 0u, 0u, 0u);
         uint4 h;
         h.x = bf16x2_to_f16x2(v.x);
         h.y = bf16x2_to_f16x2(v.y);
@@ -112,7 +114,9 @@ __device__ __forceinline__ void load_stage(Stage<RT, B>& st, const SmallM& p, in
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int row = r0 + 16 * t + g + 8 * h;
-                if (gj < ge && row < p.N) {
+                if (gj < ge && row < p.N &&
+                    Q4_IN_BOUNDS(row * rowbytes + gj * 32 + tq * 8, 8, p.N * rowbytes) &&
+                    Q4_IN_BOUNDS(static_cast<int64_t>(row) * p.G + gj, 1, static_cast<int64_t>(p.N) * p.G)) {
                     st.c[j][t][h] = ldg_stream_u2(p.codes + row * rowbytes + gj * 32 + tq * 8);
                     st.s[j][t][h] = ldg_u16(p.scales + static_cast<int64_t>(row) * p.G + gj);
                 } else {
@@ -262,7 +266,9 @@ __global__ void __launch_bounds__(kThreads, 2) small_m_kernel(const SmallM p) {
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) sum += red[(w * R + row) * p.M + m];
             const int n = r0 + row;
-            if (n < p.N) p.y[static_cast<int64_t>(m) * p.N + n] = sum;
+            if (n < p.N &&
+                Q4_IN_BOUNDS(static_cast<int64_t>(m) * p.N + n, 1, static_cast<int64_t>(p.M) * p.N))
+                p.y[static_cast<int64_t>(m) * p.N + n] = sum;
         }
         __syncthreads();
     }
@@ -327,5 +333,7 @@ cudaError_t launch_small_m(const uint8_t* codes, const uint16_t* scales, const u
     if (tiles >= 2 * slots) return launch_variant<2, 2, 2>(p, 3, s, dev);
     return launch_variant<2, 1, 4>(p, 4, s, dev);
 }
+
+Q4_DEFINE_TAKE_BOUNDS(gemv)
 
 }  // namespace q4

@@ -219,8 +219,11 @@ __device__ __forceinline__ void pass_mma(uint4 lo, uint4 hi, const uint32_t (&xr
 template <bool kEvenG>
 __device__ __forceinline__ uint32_t load_scales(const M1& p, const uint16_t* srow, int s) {
     const uint16_t* q = srow + 2 * s;
-    if (kEvenG) return ldg_u32(q);
-    return ldg_u16(q) | (ldg_u16(q + (2 * s + 1 < p.G ? 1 : 0)) << 16);
+    const long long extent = static_cast<long long>(p.N) * p.G;
+    if (kEvenG) return Q4_IN_BOUNDS(q - p.scales, 2, extent) ? ldg_u32(q) : 0u;
+    const uint16_t* q1 = q + (2 * s + 1 < p.G ? 1 : 0);
+    if (!Q4_IN_BOUNDS(q - p.scales, 1, extent) || !Q4_IN_BOUNDS(q1 - p.scales, 1, extent)) return 0u;
+    return ldg_u16(q) | (ldg_u16(q1) << 16);
 }
 
 // MT: token slots (1, 2 or 4); tokens 2 pp and 2 pp + 1 share B operand pp.
@@ -297,14 +300,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
                 if (lane == 0) {
                     const uint32_t bytes = static_cast<uint32_t>(rows * p.rowbytes);
                     mbar_arrive_expect_tx(full, bytes);
-                    bulk_load(dst, p.codes + static_cast<int64_t>(r0 + 16 * t) * p.rowbytes, bytes,
-                              full);
+                    if (Q4_IN_BOUNDS(static_cast<int64_t>(r0 + 16 * t) * p.rowbytes, bytes,
+                                     static_cast<int64_t>(p.N) * p.rowbytes))
+                        bulk_load(dst, p.codes + static_cast<int64_t>(r0 + 16 * t) * p.rowbytes, bytes,
+                                  full);
                 }
             } else {
                 const uint32_t bytes = static_cast<uint32_t>(min(p.KC, p.rowbytes - c * p.KC));
                 if (lane == 0) mbar_arrive_expect_tx(full, bytes * rows);
                 __syncwarp();
-                if (lane < rows)
+                if (lane < rows &&
+                    Q4_IN_BOUNDS(static_cast<int64_t>(r0 + 16 * t + lane) * p.rowbytes + c * p.KC, bytes,
+                                 static_cast<int64_t>(p.N) * p.rowbytes))
                     bulk_load(dst + lane * p.KC,
                               p.codes + static_cast<int64_t>(r0 + 16 * t + lane) * p.rowbytes +
                                   c * p.KC,
@@ -453,7 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                        if (act) v = ldg_v4_ordered(xs + 8 * q);
+                        if (act && Q4_IN_BOUNDS(xs + 8 * q - p.x, 8, static_cast<int64_t>(p.M) * p.K))
+                            v = ldg_v4_ordered(xs + 8 * q);
                         xw[j][pp][4 * q] = v.x;
                         xw[j][pp][4 * q + 1] = v.y;
                         xw[j][pp][4 * q + 2] = v.z;
@@ -465,8 +473,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
 #pragma unroll
             for (int i = 0; i < kXRounds; ++i) {
                 const int r = tid + i * kCW * 32;
-                xv[i] = r < nx ? __ldg(reinterpret_cast<const uint4*>(p.x) + r)
-                               : make_uint4(0u, 0u, 0u, 0u);
+                xv[i] = r < nx && Q4_IN_BOUNDS(8 * r, 8, p.K) ? __ldg(reinterpret_cast<const uint4*>(p.x) + r)
+                                                              : make_uint4(0u, 0u, 0u, 0u);
             }
         }
         asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
@@ -641,7 +649,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_m1_kernel(const M1 p) {
                 float sum = 0.f;
 #pragma unroll
                 for (int w = 0; w < kCW; ++w) sum += q[16 * MT * w];
-                p.y[static_cast<int64_t>(tok) * p.N + r0 + r] = sum;
+                if (Q4_IN_BOUNDS(static_cast<int64_t>(tok) * p.N + r0 + r, 1, static_cast<int64_t>(p.M) * p.N))
+                    p.y[static_cast<int64_t>(tok) * p.N + r0 + r] = sum;
             }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kCW * 32) : "memory");
@@ -781,5 +790,7 @@ cudaError_t launch_gemv_m1(const uint8_t* codes, const uint16_t* scales, const u
     return even ? launch_variant<true, false, false>(p, grid, smem, 20, s, dev)
                 : launch_variant<false, false, false>(p, grid, smem, 21, s, dev);
 }
+
+Q4_DEFINE_TAKE_BOUNDS(gemv_m1)
 
 }  // namespace q4

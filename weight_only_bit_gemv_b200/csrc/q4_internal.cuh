@@ -102,6 +102,48 @@ cudaError_t take_gemm_small_error(unsigned int* out);
 cudaError_t take_gemv2_error(unsigned int* out);
 
 // ---------------------------------------------------------------------------
+// bounds checks of the debug build (-DQ4_DEBUG, built as libq4_debug.so)
+// ---------------------------------------------------------------------------
+// Q4_IN_BOUNDS(first, count, extent): the elements [first, first + count) of a
+// buffer of `extent` elements all exist.  In the debug build a failed check
+// sets this translation unit's bit in its own device word and the caller skips
+// the access (a skipped bulk copy leaves its mbarrier short, so the waits
+// behind it run out and report too); nothing traps.  In the release build the
+// check is the constant true and costs nothing.
+#ifdef Q4_DEBUG
+static __device__ unsigned int g_bounds_error_tu;
+__device__ __forceinline__ bool q4_in_bounds(long long first, long long count, long long extent) {
+    const bool ok = first >= 0 && count >= 0 && first + count <= extent;
+    if (!ok) atomicOr(&g_bounds_error_tu, 1u);
+    return ok;
+}
+#define Q4_IN_BOUNDS(first, count, extent) \
+    q4::q4_in_bounds(static_cast<long long>(first), static_cast<long long>(count), static_cast<long long>(extent))
+// Copies out and clears this translation unit's word (defined once per .cu
+// file by Q4_DEFINE_TAKE_BOUNDS).
+#define Q4_DEFINE_TAKE_BOUNDS(name)                                                        \
+    cudaError_t take_bounds_##name(unsigned int* out) {                                   \
+        unsigned int zero = 0;                                                             \
+        cudaError_t e = cudaMemcpyFromSymbol(out, g_bounds_error_tu, sizeof(unsigned int)); \
+        if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_bounds_error_tu, &zero, sizeof(unsigned int)); \
+        return e;                                                                          \
+    }
+#else
+#define Q4_IN_BOUNDS(first, count, extent) true
+#define Q4_DEFINE_TAKE_BOUNDS(name)                          \
+    cudaError_t take_bounds_##name(unsigned int* out) {      \
+        *out = 0;                                            \
+        return cudaSuccess;                                  \
+    }
+#endif
+cudaError_t take_bounds_gemv_m1(unsigned int* out);
+cudaError_t take_bounds_gemm_small(unsigned int* out);
+cudaError_t take_bounds_gemm_tc(unsigned int* out);
+cudaError_t take_bounds_gemv(unsigned int* out);
+cudaError_t take_bounds_pack(unsigned int* out);
+cudaError_t take_bounds_gemv2(unsigned int* out);
+
+// ---------------------------------------------------------------------------
 // device helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

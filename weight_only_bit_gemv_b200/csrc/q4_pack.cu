@@ -48,6 +48,10 @@ __global__ void __launch_bounds__(256) pack_kernel(const float* __restrict__ w,
     for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
          idx += (int64_t)gridDim.x * blockDim.x) {
         const int64_t n = idx / G, g = idx - n * G;
+        if (!Q4_IN_BOUNDS(n * K + g * kGroup, kGroup, N * K) ||
+            !Q4_IN_BOUNDS(n * (K / 2) + g * (kGroup / 2), kGroup / 2, N * (K / 2)) ||
+            !Q4_IN_BOUNDS(n * G + g, 1, N * G))
+            continue;
         const float4* src = reinterpret_cast<const float4*>(w + n * K + g * kGroup);
         float v[kGroup];
 #pragma unroll
@@ -113,6 +117,9 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
          idx += (int64_t)gridDim.x * blockDim.x) {
         const int64_t n = idx / per_row, j = idx - n * per_row;
         const int64_t k0 = j * 16;
+        if (!Q4_IN_BOUNDS(n * (K / 2) + j * 8, 8, N * (K / 2)) || !Q4_IN_BOUNDS(n * G + k0 / kGroup, 1, N * G) ||
+            !Q4_IN_BOUNDS(n * K + k0, 16, N * K))
+            continue;
         const uint2 b = __ldg(reinterpret_cast<const uint2*>(codes + n * (K / 2) + j * 8));
         const float s = half_bits_to_float(scales[n * G + k0 / kGroup]);
         float out[16];
@@ -164,9 +171,11 @@ __global__ void __launch_bounds__(256) embed_rows_kernel(const uint8_t* __restri
          idx += (int64_t)gridDim.x * blockDim.x) {
         const int64_t i = idx / per_row, j = idx - i * per_row;
         const int64_t k0 = j * 16;
+        if (!Q4_IN_BOUNDS(i, 1, n_ids) || !Q4_IN_BOUNDS(i * K + k0, 16, n_ids * K)) continue;
         const int64_t n = __ldg(ids + i);
         float v[16];
-        if (n >= 0 && n < N) {
+        if (n >= 0 && n < N && Q4_IN_BOUNDS(n * (K / 2) + j * 8, 8, N * (K / 2)) &&
+            Q4_IN_BOUNDS(n * G + k0 / kGroup, 1, N * G)) {
             const uint2 b = __ldg(reinterpret_cast<const uint2*>(codes + n * (K / 2) + j * 8));
             const float sc = half_bits_to_float(scales[n * G + k0 / kGroup]);
 #pragma unroll
@@ -201,5 +210,7 @@ cudaError_t launch_embed_rows(const uint8_t* codes, const uint16_t* scales, cons
                                                                K);
     return cudaGetLastError();
 }
+
+Q4_DEFINE_TAKE_BOUNDS(pack)
 
 }  // namespace q4
