@@ -521,7 +521,7 @@ __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
             const int cbytes = kWhole ? p.R : min(p.KC, p.R - c * p.KC);
             if (lane == 0) mbar_arrive_expect_tx(full, static_cast<uint32_t>(rows * cbytes));
             __syncwarp();
-            const int64_t code_extent = static_cast<int64_t>(p.N) * p.R;
+            [[maybe_unused]] const int64_t code_extent = static_cast<int64_t>(p.N) * p.R;
             if (kWhole) {
                 if (lane == 0 && Q4_IN_BOUNDS(static_cast<int64_t>(row0) * p.R, rows * p.R, code_extent))
                     bulk_load(dst, p.codes + static_cast<int64_t>(row0) * p.R, static_cast<uint32_t>(rows * p.R), full);

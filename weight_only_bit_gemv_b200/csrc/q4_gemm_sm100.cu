@@ -43,6 +43,7 @@
 // which measured 1.2-1.3x faster at M = 40-128.
 // Every wait is bounded; a timeout sets an error bit, the roles drain what
 // they have in flight and the CTA frees its tensor memory before it exits.
+#include <algorithm>
 #include <mutex>
 
 #include "q4_internal.cuh"
@@ -82,12 +83,63 @@ struct TcGemm {
     int M, N, K, G;
     int BMT;            // tokens per tile (MMA N), multiple of 16, <= 256
     int token_tiles;    // ceil(M / BMT)
-    int ksplit;         // K chunks per tile
-    int chunk_groups;   // groups per K chunk (multiple of kWG)
+    int tiles;          // (strip groups of kStrips strips) x token tiles; tile t = sp * token_tiles + tt
+    int W;              // weight stages (kWG groups) per tile: ceil(G / kWG)
+    int full;           // stream-K plan: whole tiles per CTA, taken first
+    int ks;             // chunk plan (ks >= 1): each tile in ks chunks of cw stages; 0: stream-K plan
+    int cw;
     int xstages;
     int xstage_bytes;   // BMT * 128
     int wscale_off, x_off, cb_off, bar_off;
     uint32_t idesc;
+};
+
+// The work of one CTA (persistent, one per SM), in order.  Stream-K plan
+// (ks == 0): `full` whole tiles (tile i * gridDim.x + blockIdx.x), then an
+// even share of the weight stages of the tiles left over: units u over those
+// tiles, tile full * gridDim.x + u / W, stage u mod W.  Chunk plan (ks >= 1):
+// chunks v = blockIdx.x + i * gridDim.x of the tiles x ks chunks, chunk v
+// being stages [cw (v mod ks), +cw) of tile v / ks.  A segment is stages
+// [w0, w1) of one tile; it is whole when it covers every stage, and is then
+// stored plainly, else added (red.add) into y that the x conversion zeroed.
+struct Seg {
+    int tile, w0, w1;
+};
+struct SegCursor {
+    int k;
+    long long u, u1;
+    __device__ explicit SegCursor(const TcGemm& p) : k(0) {
+        const long long ru =
+            static_cast<long long>(p.tiles - p.full * static_cast<int>(gridDim.x)) * p.W;
+        u = ru * blockIdx.x / gridDim.x;
+        u1 = ru * (blockIdx.x + 1) / gridDim.x;
+    }
+    __device__ bool next(const TcGemm& p, Seg& sg) {
+        if (p.ks > 0) {
+            const long long v = static_cast<long long>(k) * gridDim.x + blockIdx.x;
+            if (v >= static_cast<long long>(p.tiles) * p.ks) return false;
+            sg.tile = static_cast<int>(v / p.ks);
+            sg.w0 = static_cast<int>(v % p.ks) * p.cw;
+            sg.w1 = sg.w0 + p.cw < p.W ? sg.w0 + p.cw : p.W;
+            ++k;
+            return true;
+        }
+        if (k < p.full) {
+            sg.tile = k * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x);
+            sg.w0 = 0;
+            sg.w1 = p.W;
+            ++k;
+            return true;
+        }
+        if (u >= u1) return false;
+        const long long t = u / p.W;
+        sg.tile = p.full * static_cast<int>(gridDim.x) + static_cast<int>(t);
+        sg.w0 = static_cast<int>(u - t * p.W);
+        const long long left = u1 - u;
+        sg.w1 = left < p.W - sg.w0 ? sg.w0 + static_cast<int>(left) : p.W;
+        u += sg.w1 - sg.w0;
+        return true;
+    }
 };
 
 __device__ __forceinline__ void named_sync(int id, int threads) {
@@ -124,27 +176,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t base = smem_u32(smem);
     const uint32_t bars = base + p.bar_off;
-    // barriers: wfull, wempty [kWStages]; xfull, afull, gdone [kASlots]; dfull, cbbar, drain
+    // barriers: wfull, wempty [kWStages]; xfull, afull, gdone [kASlots];
+    // afilled, cbbar, drain, aempty
     auto wfull = [&](int s) { return bars + 8u * s; };
     auto wempty = [&](int s) { return bars + 8u * (kWStages + s); };
     auto xfull = [&](int s) { return bars + 8u * (2 * kWStages + s); };
     auto afull = [&](int s) { return bars + 8u * (2 * kWStages + kASlots + s); };
     auto gdone = [&](int s) { return bars + 8u * (2 * kWStages + 2 * kASlots + s); };
-    const uint32_t dfull = bars + 8u * (2 * kWStages + 3 * kASlots);
-    const uint32_t cbbar = dfull + 8u;
-    const uint32_t drain = dfull + 16u;
+    const uint32_t afilled = bars + 8u * (2 * kWStages + 3 * kASlots);  // accumulator complete
+    const uint32_t cbbar = afilled + 8u;
+    const uint32_t drain = afilled + 16u;
+    const uint32_t aempty = afilled + 24u;  // accumulator read out by the epilogue
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + p.cb_off + 32);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + p.cb_off + 36);
-
-    // tile coordinates: blockIdx.x = ((tile * token_tiles) + tt) * ksplit + kc;
-    // the tile's first strip is kStrips * tile
-    const int kc = blockIdx.x % p.ksplit;
-    const int tt = (blockIdx.x / p.ksplit) % p.token_tiles;
-    const int strip = kStrips * (blockIdx.x / (p.ksplit * p.token_tiles));
-    const int g_begin = kc * p.chunk_groups;
-    const int g_end = min(p.G, g_begin + p.chunk_groups);
-    const int ng = g_end - g_begin;  // groups of this CTA, >= 1
-    const int nw = (ng + kWG - 1) / kWG;
 
     if (tid == 0) {
         for (int s = 0; s < kWStages; ++s) {
@@ -156,9 +200,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(afull(s), 4);   // the four warps of the owning warpgroup
             mbar_init(gdone(s), 1);   // tcgen05.commit after the group's MMAs
         }
-        mbar_init(dfull, 1);
+        mbar_init(afilled, 1);
         mbar_init(cbbar, 1);
         mbar_init(drain, 1);
+        mbar_init(aempty, kDecWarps);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -178,50 +223,56 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(cbbar, 32u);
             bulk_load(base + p.cb_off, p.cb, 32u, cbbar);
         }
-        int wi = 0;  // weight stages issued
+        int wi = 0;  // weight stages issued, over all segments
         bool ok = true;
-        for (int w = 0; w < nw && ok; ++w) {
-            // weight stage w: groups g_begin + 4w .. +3
-            const int ws = w % kWStages;
-            if (w >= kWStages && !warp_wait(wempty(ws), static_cast<uint32_t>(w / kWStages - 1) & 1u, lane)) {
-                ok = false;
-                break;
-            }
-            const int g0 = g_begin + kWG * w;
-            const uint32_t cdst = base + kLutBytes + ws * kStageCode;
-            const uint32_t sdst = base + p.wscale_off + ws * kStageScale;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(wfull(ws), kStageCode);
+        SegCursor cur(p);
+        Seg sg;
+        while (ok && cur.next(p, sg)) {
+            const int strip = kStrips * (sg.tile / p.token_tiles);
+            for (int w = sg.w0; w < sg.w1; ++w, ++wi) {
+                // weight stage w of the tile: groups 4w .. min(G, 4w + 4) - 1
+                const int ws = wi % kWStages;
+                if (wi >= kWStages &&
+                    !warp_wait(wempty(ws), static_cast<uint32_t>(wi / kWStages - 1) & 1u, lane)) {
+                    ok = false;
+                    break;
+                }
+                const int g0 = kWG * w;
+                const int g_end = min(p.G, g0 + kWG);
+                const uint32_t cdst = base + kLutBytes + ws * kStageCode;
+                const uint32_t sdst = base + p.wscale_off + ws * kStageScale;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(wfull(ws), kStageCode);
 #pragma unroll
-                for (int h = 0; h < kStrips; ++h)
-                    tma_load_2d(cdst + h * kWCodeBytes, &cmap, g0 * 32, (strip + h) * kR, wfull(ws));
-            }
+                    for (int h = 0; h < kStrips; ++h)
+                        tma_load_2d(cdst + h * kWCodeBytes, &cmap, g0 * 32, (strip + h) * kR, wfull(ws));
+                }
 #pragma unroll
-            for (int jr = 0; jr < kStrips * kR / 32; ++jr) {
-                const int r = lane + 32 * jr;
-                const int row = strip * kR + r;
-                if (kAsyncScales) {
-                    const bool in = row < p.N && Q4_IN_BOUNDS(static_cast<long long>(row) * p.G + g0, 4,
-                                                              static_cast<long long>(p.N) * p.G);
-                    const uint16_t* src = in ? p.scales + static_cast<long long>(row) * p.G + g0 : p.scales;
-                    cp_async_8(sdst + r * 8, src, in ? 8u : 0u);
-                } else {
+                for (int jr = 0; jr < kStrips * kR / 32; ++jr) {
+                    const int r = lane + 32 * jr;
+                    const int row = strip * kR + r;
+                    if (kAsyncScales) {
+                        const bool in = row < p.N && Q4_IN_BOUNDS(static_cast<long long>(row) * p.G + g0, 4,
+                                                                  static_cast<long long>(p.N) * p.G);
+                        const uint16_t* src = in ? p.scales + static_cast<long long>(row) * p.G + g0 : p.scales;
+                        cp_async_8(sdst + r * 8, src, in ? 8u : 0u);
+                    } else {
 #pragma unroll
-                    for (int q = 0; q < kWG; ++q) {
-                        uint16_t v = 0;
-                        if (row < p.N && g0 + q < g_end &&
-                            Q4_IN_BOUNDS(static_cast<long long>(row) * p.G + g0 + q, 1,
-                                         static_cast<long long>(p.N) * p.G))
-                            v = p.scales[static_cast<long long>(row) * p.G + g0 + q];
-                        sts_u16(sdst + r * 8 + 2 * q, v);
+                        for (int q = 0; q < kWG; ++q) {
+                            uint16_t v = 0;
+                            if (row < p.N && g0 + q < g_end &&
+                                Q4_IN_BOUNDS(static_cast<long long>(row) * p.G + g0 + q, 1,
+                                             static_cast<long long>(p.N) * p.G))
+                                v = p.scales[static_cast<long long>(row) * p.G + g0 + q];
+                            sts_u16(sdst + r * 8 + 2 * q, v);
+                        }
                     }
                 }
+                if (kAsyncScales)
+                    cp_async_arrive_noinc(wfull(ws));
+                else
+                    mbar_arrive(wfull(ws));
             }
-            if (kAsyncScales)
-                cp_async_arrive_noinc(wfull(ws));
-            else
-                mbar_arrive(wfull(ws));
-            ++wi;
         }
         if (!ok && lane == 0) {
             atomicOr(&g_gemm_tc_error, 1u);
@@ -232,25 +283,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!warp_wait(wfull(i % kWStages), static_cast<uint32_t>(i / kWStages) & 1u, lane)) break;
     } else if (warp == kXWarp) {
         // ----------------------------- x producer -----------------------------
-        // x tile of group gi -> ring slot gi mod kASlots, reused once the
-        // MMAs of group gi - kASlots are done.
+        // x tile of the CTA's group gi (counted over all segments) -> ring
+        // slot gi mod kASlots, reused once the MMAs of group gi - kASlots are done.
         if (lane == 0) prefetch_tensor_map(&xmap);
         int xi = 0;
-        bool ok = true;
-        for (; xi < ng; ++xi) {
-            const int xs = xi % kASlots;
-            if (xi >= kASlots &&
-                !warp_wait(gdone(xs), static_cast<uint32_t>(xi / kASlots - 1) & 1u, lane)) {
-                ok = false;
-                break;
+        bool ok = true, stop = false;
+        SegCursor cur(p);
+        Seg sg;
+        while (ok && !stop && cur.next(p, sg)) {
+            const int tt = sg.tile % p.token_tiles;
+            const int g_hi = min(p.G, kWG * sg.w1);
+            for (int g = kWG * sg.w0; g < g_hi; ++g, ++xi) {
+                const int xs = xi % kASlots;
+                if (xi >= kASlots &&
+                    !warp_wait(gdone(xs), static_cast<uint32_t>(xi / kASlots - 1) & 1u, lane)) {
+                    ok = false;
+                    break;
+                }
+                if (__shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) {
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(xfull(xs), static_cast<uint32_t>(p.xstage_bytes));
+                    tma_load_2d(base + p.x_off + xs * p.xstage_bytes, &xmap, g * 64, tt * p.BMT, xfull(xs));
+                }
+                __syncwarp();
             }
-            if (__shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(xfull(xs), static_cast<uint32_t>(p.xstage_bytes));
-                tma_load_2d(base + p.x_off + xs * p.xstage_bytes, &xmap, (g_begin + xi) * 64, tt * p.BMT,
-                            xfull(xs));
-            }
-            __syncwarp();
         }
         if (!ok && lane == 0) {
             atomicOr(&g_gemm_tc_error, 4u);
@@ -260,26 +319,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!warp_wait(xfull(i % kASlots), static_cast<uint32_t>(i / kASlots) & 1u, lane)) break;
     } else if (warp == 1) {
         // -------------------------------- MMA ---------------------------------
+        // Per segment: wait until the epilogue has read the accumulator of the
+        // previous one, then per group four MMAs (the first overwrites the
+        // accumulator), one commit that frees the group's A slot and x stage,
+        // and at the end a commit that hands the accumulator to the epilogue.
         if (lane == 0) {
             bool ok = true;
-            for (int gi = 0; gi < ng && ok; ++gi) {
-                const int as = gi % kASlots;
-                if (!mbar_wait(afull(as), static_cast<uint32_t>(gi / kASlots) & 1u) ||
-                    !mbar_wait(xfull(as), static_cast<uint32_t>(gi / kASlots) & 1u) || *abort_flag) {
+            int gi = 0, si = 0;
+            SegCursor cur(p);
+            Seg sg;
+            while (ok && cur.next(p, sg)) {
+                if (si > 0 && !mbar_wait(aempty, static_cast<uint32_t>(si - 1) & 1u)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
-                const uint64_t bd = smem_desc_sw128(base + p.x_off + as * p.xstage_bytes, 1024);
+                const int ng = min(p.G, kWG * sg.w1) - kWG * sg.w0;
+                for (int k = 0; k < ng; ++k, ++gi) {
+                    const int as = gi % kASlots;
+                    if (!mbar_wait(afull(as), static_cast<uint32_t>(gi / kASlots) & 1u) ||
+                        !mbar_wait(xfull(as), static_cast<uint32_t>(gi / kASlots) & 1u) || *abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t bd = smem_desc_sw128(base + p.x_off + as * p.xstage_bytes, 1024);
 #pragma unroll
-                for (int h = 0; h < kStrips; ++h)
+                    for (int h = 0; h < kStrips; ++h)
 #pragma unroll
-                    for (int t = 0; t < 4; ++t)
-                        tc_mma_ts(tmem + 128u * h, tmem + a_col<kStrips>(as, h) + 8 * t, bd + 2 * t,
-                                  p.idesc, (gi > 0 || t > 0) ? 1u : 0u);
-                tc_commit(gdone(as));  // frees the A slot and the x stage
+                        for (int t = 0; t < 4; ++t)
+                            tc_mma_ts(tmem + 128u * h, tmem + a_col<kStrips>(as, h) + 8 * t, bd + 2 * t,
+                                      p.idesc, (k > 0 || t > 0) ? 1u : 0u);
+                    tc_commit(gdone(as));  // frees the A slot and the x stage
+                }
+                if (!ok) break;
+                tc_commit(afilled);
+                ++si;
             }
-            if (ok) tc_commit(dfull);
             if (!ok) {
                 atomicOr(&g_gemm_tc_error, 2u);
                 *abort_flag = 1;
@@ -305,86 +380,128 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         named_sync(2, kDecWarps * 32);  // table ready
 
-        // warpgroup wg decodes groups gi = wg, wg + 2, ... into A slots gi mod 4
-        for (int gi = wg; gi < ng && ok; gi += 2) {
-            const int w = gi / kWG, ws = w % kWStages, j = gi % kWG;
-            const int as = gi % kASlots;
-            if (!warp_wait(wfull(ws), static_cast<uint32_t>(w / kWStages) & 1u, lane) ||
-                __shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) {
-                ok = false;
-                break;
-            }
-            if (gi >= kASlots && !warp_wait(gdone(as), static_cast<uint32_t>(gi / kASlots - 1) & 1u, lane)) {
-                ok = false;
-                break;
-            }
-            const int r8 = row & 7;
-#pragma unroll
+        // Epilogue of segment `si`: each warpgroup writes half of the
+        // accumulator columns.  Columns come out of tensor memory 64 at a
+        // time (two loads, one wait).  Whole tiles are stored, parts of a
+        // split tile added.
+        auto epilogue = [&](const Seg& e, int si) -> bool {
+            if (!warp_wait(afilled, static_cast<uint32_t>(si) & 1u, lane)) return false;
+            tc_fence_after();
+            const int tt = e.tile % p.token_tiles;
+            const int strip = kStrips * (e.tile / p.token_tiles);
+            const bool add = !(e.w0 == 0 && e.w1 == p.W);
+            const int half = p.BMT / 2;
+            const int c_beg = wg * half, c_end = (wg + 1) * half;
             for (int hs = 0; hs < kStrips; ++hs) {
-                const uint32_t rb = kLutBytes + ws * kStageCode + hs * kWCodeBytes + row * 128;
-                const uint4 c0 = ld_smem<uint4>(smem, rb + (((2 * j) ^ r8) << 4));
-                const uint4 c1 = ld_smem<uint4>(smem, rb + (((2 * j + 1) ^ r8) << 4));
-                const uint32_t sb = ld_smem<uint16_t>(
-                    smem, p.wscale_off + ws * kStageScale + hs * kWScaleBytes + row * 8 + 2 * j);
-                const uint32_t s2 = sb | (sb << 16);
-                const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                uint32_t h[32];
+                const int n = (strip + hs) * kR + row;
+                const uint32_t tcol = tlane + 128u * hs;
+                auto put = [&](int c, uint32_t bits) {
+                    const int m = tt * p.BMT + c;
+                    if (n < p.N && m < p.M &&
+                        Q4_IN_BOUNDS(static_cast<long long>(m) * p.N + n, 1, static_cast<long long>(p.M) * p.N)) {
+                        float* dst = p.y + static_cast<long long>(m) * p.N + n;
+                        if (add)
+                            red_add_f32(dst, __uint_as_float(bits));
+                        else
+                            *dst = __uint_as_float(bits);
+                    }
+                };
+                int c0 = c_beg;
+                for (; c0 + 64 <= c_end; c0 += 64) {
+                    uint32_t v[64];
+                    tc_ld_x32(tcol + c0, v);
+                    tc_ld_x32(tcol + c0 + 32, v + 32);
+                    tc_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    h[4 * i + 0] = hmul2_u32(lut_at<0>(smem, wd[i], lane4), s2);
-                    h[4 * i + 1] = hmul2_u32(lut_at<1>(smem, wd[i], lane4), s2);
-                    h[4 * i + 2] = hmul2_u32(lut_at<2>(smem, wd[i], lane4), s2);
-                    h[4 * i + 3] = hmul2_u32(lut_at<3>(smem, wd[i], lane4), s2);
+                    for (int i = 0; i < 64; ++i) put(c0 + i, v[i]);
                 }
-                tc_st_x32(tlane + a_col<kStrips>(as, hs), h);
+                for (; c0 + 32 <= c_end; c0 += 32) {
+                    uint32_t v[32];
+                    tc_ld_x32(tcol + c0, v);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) put(c0 + i, v[i]);
+                }
+                for (; c0 < c_end; c0 += 8) {
+                    uint32_t v[8];
+                    tc_ld_x8(tcol + c0, v);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) put(c0 + i, v[i]);
+                }
             }
-            tc_wait_st();
+            // the accumulator may now be overwritten by the next segment's MMAs
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(afull(as));
-            // this warpgroup's last group of the weight stage releases it
-            const bool last_in_stage = (j + 2 >= kWG) || (gi + 2 >= ng);
-            if (last_in_stage) {
+            if (lane == 0) mbar_arrive(aempty);
+            return true;
+        };
+
+        // Stage by stage: warpgroup wg decodes the stage's groups j = wg,
+        // wg + 2 into A slots (CTA group index) mod 4; both warpgroups
+        // release every stage they waited for.
+        int gi = 0, wi = 0, si = 0;
+        bool epi_ok = true;
+        SegCursor cur(p);
+        Seg sg, prev{0, 0, 0};
+        while (ok && cur.next(p, sg)) {
+            if (si > 0 && !(epi_ok = epilogue(prev, si - 1))) break;
+            for (int w = sg.w0; w < sg.w1; ++w, ++wi) {
+                const int ws = wi % kWStages;
+                if (!warp_wait(wfull(ws), static_cast<uint32_t>(wi / kWStages) & 1u, lane) ||
+                    __shfl_sync(0xFFFFFFFFu, *abort_flag, 0)) {
+                    ok = false;
+                    break;
+                }
+                const int gs = min(kWG, p.G - kWG * w);  // groups in this stage
+                const int r8 = row & 7;
+                for (int j = wg; j < gs; j += 2) {
+                    const int g = gi + j, as = g % kASlots;
+                    if (g >= kASlots &&
+                        !warp_wait(gdone(as), static_cast<uint32_t>(g / kASlots - 1) & 1u, lane)) {
+                        ok = false;
+                        break;
+                    }
+#pragma unroll
+                    for (int hs = 0; hs < kStrips; ++hs) {
+                        const uint32_t rb = kLutBytes + ws * kStageCode + hs * kWCodeBytes + row * 128;
+                        const uint4 c0 = ld_smem<uint4>(smem, rb + (((2 * j) ^ r8) << 4));
+                        const uint4 c1 = ld_smem<uint4>(smem, rb + (((2 * j + 1) ^ r8) << 4));
+                        const uint32_t sb = ld_smem<uint16_t>(
+                            smem, p.wscale_off + ws * kStageScale + hs * kWScaleBytes + row * 8 + 2 * j);
+                        const uint32_t s2 = sb | (sb << 16);
+                        const uint32_t wd[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                        uint32_t h[32];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            h[4 * i + 0] = hmul2_u32(lut_at<0>(smem, wd[i], lane4), s2);
+                            h[4 * i + 1] = hmul2_u32(lut_at<1>(smem, wd[i], lane4), s2);
+                            h[4 * i + 2] = hmul2_u32(lut_at<2>(smem, wd[i], lane4), s2);
+                            h[4 * i + 3] = hmul2_u32(lut_at<3>(smem, wd[i], lane4), s2);
+                        }
+                        tc_st_x32(tlane + a_col<kStrips>(as, hs), h);
+                    }
+                    tc_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(afull(as));
+                }
+                if (!ok) break;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(wempty(ws));
+                gi += gs;
             }
+            prev = sg;
+            ++si;
         }
+        if (ok && epi_ok && si > 0) epi_ok = epilogue(prev, si - 1);
         if (!ok && lane == 0) {
             atomicOr(&g_gemm_tc_error, 8u);
             *abort_flag = 1;
         }
-        // epilogue: each warpgroup writes half of the accumulator columns
-        if (warp_wait(dfull, 0u, lane)) {
-            tc_fence_after();
-            const int half = p.BMT / 2;
-            for (int hs = 0; hs < kStrips; ++hs) {
-                const int n = (strip + hs) * kR + row;
-                for (int c0 = wg * half; c0 < (wg + 1) * half; c0 += 8) {
-                    uint32_t v[8];
-                    asm volatile(
-                        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-                        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
-                          "=r"(v[6]), "=r"(v[7])
-                        : "r"(tlane + 128u * hs + c0)
-                        : "memory");
-                    tc_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int m = tt * p.BMT + c0 + e;
-                        if (n < p.N && m < p.M &&
-                            Q4_IN_BOUNDS(static_cast<long long>(m) * p.N + n, 1,
-                                         static_cast<long long>(p.M) * p.N)) {
-                            float* dst = p.y + static_cast<long long>(m) * p.N + n;
-                            if (p.ksplit > 1)
-                                red_add_f32(dst, __uint_as_float(v[e]));
-                            else
-                                *dst = __uint_as_float(v[e]);
-                        }
-                    }
-                }
-            }
-        } else if (lane == 0) {
+        if (!epi_ok && lane == 0) {
             atomicOr(&g_gemm_tc_error, 32u);
+            *abort_flag = 1;
         }
     }
 
@@ -397,9 +514,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// xh_elems: binary16 elements the destination array holds
+// The tiles whose segments are added into y rather than stored: y of tiles
+// [first, first + count) is zeroed before the GEMM runs.  Tile t covers rows
+// [rows * (t / token_tiles), +rows) and tokens [BMT * (t % token_tiles), +BMT).
+struct ZeroTiles {
+    float* y;
+    int M, N, BMT, token_tiles, rows;
+    int first, count;
+};
+
+// x -> binary16 (xh_elems: elements the destination array holds), then the
+// zeroing of the added tiles' outputs.
 __global__ void bf16_to_f16_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ xh, int64_t n8,
-                                   int64_t xh_elems) {
+                                   int64_t xh_elems, const ZeroTiles z) {
+    const int64_t per_tile = static_cast<int64_t>(z.BMT) * z.rows;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < z.count * per_tile;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int t = z.first + static_cast<int>(i / per_tile);
+        const int r = static_cast<int>(i % per_tile);
+        const int m = (t % z.token_tiles) * z.BMT + r / z.rows;
+        const int n = (t / z.token_tiles) * z.rows + r % z.rows;
+        if (m < z.M && n < z.N &&
+            Q4_IN_BOUNDS(static_cast<int64_t>(m) * z.N + n, 1, static_cast<int64_t>(z.M) * z.N))
+            z.y[static_cast<int64_t>(m) * z.N + n] = 0.0f;
+    }
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         if (!Q4_IN_BOUNDS(8 * i, 8, xh_elems)) continue;
@@ -441,25 +579,72 @@ cudaError_t launch_prefill_tc(const uint8_t* codes, const uint16_t* scales, cons
     // two strips per tile share each x tile when both accumulators fit
     // (2 x BMT <= 256 tensor-memory columns)
     const int nstrips = p.BMT <= 128 ? 2 : 1;
-    const int tiles = (strips + nstrips - 1) / nstrips * p.token_tiles;
-    // K split: fewest waves x longest chunk (plus a fixed cost of ~4 groups),
-    // one CTA per SM; ties go to the smaller split
-    int ksplit = 1, chunk = (p.G + kWG - 1) / kWG * kWG;
-    long long best = -1;
-    for (int ks = 1; ks <= (p.G + kWG - 1) / kWG; ++ks) {
-        const int c = ((p.G + ks - 1) / ks + kWG - 1) / kWG * kWG;
-        const int real = (p.G + c - 1) / c;
-        if (real != ks) continue;
-        const long long waves = (static_cast<long long>(tiles) * ks + dev.sm_count - 1) / dev.sm_count;
-        const long long cost = waves * (c + 4);
-        if (best < 0 || cost < best) {
+    p.tiles = (strips + nstrips - 1) / nstrips * p.token_tiles;
+    p.W = (p.G + kWG - 1) / kWG;
+    // Persistent CTAs, one per SM at most.  Two kinds of plan: stream-K (each
+    // CTA takes `full` whole tiles, then an even share of the stages of the
+    // tiles left over) and chunks (each tile cut into ks chunks of K, dealt
+    // out round-robin).  The cheaper by a cost model measured on B200 with
+    // the Llama-2-70B shapes at 32-512 tokens: a weight stage takes
+    // 4 x max(0.42 BMT kStrips / 256, 0.12 kStrips) us, each segment a
+    // further 2.5 us plus 5.5 us per 128 KB of its tile's outputs (pipeline
+    // restart and epilogue, the MMAs idle meanwhile), zeroing y at ~5 TB/s
+    // and red.add at ~4 TB/s.  Stream-K wins when most work is in whole
+    // tiles; with fewer tiles than SMs, chunks of equal size usually do.
+    const double ts = 4.0 * std::max(0.42 * p.BMT * nstrips / 256.0, 0.12 * nstrips);
+    const double tile_bytes = 4.0 * p.BMT * nstrips * kR;
+    const double te = 2.5 + 5.5 * tile_bytes / 131072.0;
+    const double zbw = 5.0e3, rbw = 4.0e3;  // bytes per ns
+    const long long units = static_cast<long long>(p.tiles) * p.W;
+    int grid = 1;
+    double best = -1.0;
+    {
+        // stream-K
+        long long g64 = units / 2 > 0 ? units / 2 : 1;
+        if (g64 > dev.sm_count) g64 = dev.sm_count;
+        const int gs = static_cast<int>(g64);
+        const int full = p.tiles / gs;
+        const long long ru = static_cast<long long>(p.tiles - full * gs) * p.W;
+        double worst = 0.0, adds = 0.0;
+        for (int c = 0; c < gs; ++c) {
+            long long u = ru * c / gs;
+            const long long u1 = ru * (c + 1) / gs;
+            int segs = 0;
+            for (; u < u1; ++segs) {
+                const long long w0 = u % p.W;
+                u += std::min<long long>(u1 - u, p.W - w0);
+            }
+            adds += segs;
+            const double cost = full * (p.W * ts + te) + (u1 - ru * c / gs) * ts + segs * te;
+            worst = std::max(worst, cost);
+        }
+        const double cost = worst + (p.tiles - full * gs) * tile_bytes / (zbw * 1e3) +
+                            adds * tile_bytes / (rbw * 1e3);
+        best = cost;
+        grid = gs;
+        p.full = full;
+        p.ks = 0;
+        p.cw = 0;
+    }
+    for (int ks = 1; ks <= 8 && ks <= p.W; ++ks) {
+        const int cw = (p.W + ks - 1) / ks;
+        if ((p.W + cw - 1) / cw != ks) continue;
+        const long long vt = static_cast<long long>(p.tiles) * ks;
+        const int gk = static_cast<int>(std::min<long long>(vt, dev.sm_count));
+        const long long rounds = (vt + gk - 1) / gk;
+        double cost = rounds * (cw * ts + te);
+        if (ks > 1) {
+            const double ybytes = 4.0 * static_cast<double>(M) * static_cast<double>(N);
+            cost += ybytes / (zbw * 1e3) + ks * ybytes / (rbw * 1e3);
+        }
+        if (cost < best) {
             best = cost;
-            ksplit = ks;
-            chunk = c;
+            grid = gk;
+            p.full = 0;
+            p.ks = ks;
+            p.cw = cw;
         }
     }
-    p.ksplit = ksplit;
-    p.chunk_groups = chunk;
     p.xstage_bytes = p.BMT * 128;
     p.idesc = idesc_f16_f32(kR, p.BMT);
     p.wscale_off = kLutBytes + kWStages * nstrips * kWCodeBytes;
@@ -468,16 +653,38 @@ cudaError_t launch_prefill_tc(const uint8_t* codes, const uint16_t* scales, cons
     p.xstages = SX;
     p.cb_off = p.x_off + SX * p.xstage_bytes;
     p.bar_off = p.cb_off + 64;
-    const int nbars = 2 * kWStages + 3 * kASlots + 3;
+    const int nbars = 2 * kWStages + 3 * kASlots + 4;
     const int smem = p.bar_off + nbars * 8;
     if (smem > dev.smem_optin) return cudaErrorNotSupported;
 
     // x -> binary16 into the scratch buffer
     const int64_t n8 = M * K / 8;
-    int cgrid = static_cast<int>((n8 + 255) / 256);
+    const int zero_tiles = p.ks == 0 ? p.tiles - p.full * grid : (p.ks > 1 ? p.tiles : 0);
+    const int64_t zero_elems =
+        zero_tiles == p.tiles ? 0 : static_cast<int64_t>(zero_tiles) * p.BMT * nstrips * kR;
+    const int64_t work = n8 > zero_elems ? n8 : zero_elems;
+    int cgrid = static_cast<int>((work + 255) / 256);
     if (cgrid > dev.sm_count * 8) cgrid = dev.sm_count * 8;
-    bf16_to_f16_kernel<<<cgrid, 256, 0, s>>>(x, xh, n8, xh_elems);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = cudaSuccess;
+    ZeroTiles z{};
+    z.y = y;
+    z.M = p.M;
+    z.N = p.N;
+    z.BMT = p.BMT;
+    z.token_tiles = p.token_tiles;
+    z.rows = nstrips * kR;
+    // tiles whose segments are added: the leftover tiles of stream-K, every
+    // tile of a plan in several chunks.  When that is all of y, one memset
+    // (faster than the conversion kernel's scalar stores) zeroes it.
+    z.first = p.ks == 0 ? p.full * grid : 0;
+    z.count = zero_tiles;
+    if (zero_tiles == p.tiles) {
+        e = cudaMemsetAsync(y, 0, static_cast<size_t>(M) * N * sizeof(float), s);
+        if (e != cudaSuccess) return e;
+        z.count = 0;
+    }
+    bf16_to_f16_kernel<<<cgrid, 256, 0, s>>>(x, xh, n8, xh_elems, z);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
     CUtensorMap cmap, xmap;
@@ -489,10 +696,6 @@ cudaError_t launch_prefill_tc(const uint8_t* codes, const uint16_t* scales, cons
                              static_cast<uint64_t>(K), static_cast<uint64_t>(K) * 2, p.BMT, 64,
                              CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
-    if (ksplit > 1) {
-        e = cudaMemsetAsync(y, 0, static_cast<size_t>(M) * N * sizeof(float), s);
-        if (e != cudaSuccess) return e;
-    }
     const bool async_scales = (p.G % kWG) == 0;
     const void* fn = nstrips == 2
                          ? (async_scales ? reinterpret_cast<const void*>(gemm_tc_kernel<true, 2>)
@@ -501,7 +704,6 @@ cudaError_t launch_prefill_tc(const uint8_t* codes, const uint16_t* scales, cons
                                          : reinterpret_cast<const void*>(gemm_tc_kernel<false, 1>));
     e = ensure_smem_attr(fn, smem, 30 + (async_scales ? 0 : 1) + 2 * (nstrips - 1), dev.device);
     if (e != cudaSuccess) return e;
-    const int grid = tiles * ksplit;
     if (nstrips == 2) {
         if (async_scales)
             gemm_tc_kernel<true, 2><<<grid, kThreads, smem, s>>>(cmap, xmap, p);

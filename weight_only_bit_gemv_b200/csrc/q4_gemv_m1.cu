@@ -219,7 +219,7 @@ __device__ __forceinline__ void pass_mma(uint4 lo, uint4 hi, const uint32_t (&xr
 template <bool kEvenG>
 __device__ __forceinline__ uint32_t load_scales(const M1& p, const uint16_t* srow, int s) {
     const uint16_t* q = srow + 2 * s;
-    const long long extent = static_cast<long long>(p.N) * p.G;
+    [[maybe_unused]] const long long extent = static_cast<long long>(p.N) * p.G;
     if (kEvenG) return Q4_IN_BOUNDS(q - p.scales, 2, extent) ? ldg_u32(q) : 0u;
     const uint16_t* q1 = q + (2 * s + 1 < p.G ? 1 : 0);
     if (!Q4_IN_BOUNDS(q - p.scales, 1, extent) || !Q4_IN_BOUNDS(q1 - p.scales, 1, extent)) return 0u;
