@@ -381,9 +381,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_sync(2, kDecWarps * 32);  // table ready
 
         // Epilogue of segment `si`: each warpgroup writes half of the
-        // accumulator columns.  Columns come out of tensor memory 64 at a
-        // time (two loads, one wait).  Whole tiles are stored, parts of a
-        // split tile added.
+        // accumulator columns, 8 at a time, in a rolled loop (as fast on B200
+        // as a 64-column unrolled body, and a fraction of the code).  Whole
+        // tiles are stored, parts of a split tile added.
         auto epilogue = [&](const Seg& e, int si) -> bool {
             if (!warp_wait(afilled, static_cast<uint32_t>(si) & 1u, lane)) return false;
             tc_fence_after();
@@ -391,43 +391,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int strip = kStrips * (e.tile / p.token_tiles);
             const bool add = !(e.w0 == 0 && e.w1 == p.W);
             const int half = p.BMT / 2;
-            const int c_beg = wg * half, c_end = (wg + 1) * half;
+            const int m_beg = tt * p.BMT + wg * half;
+            // columns of this warpgroup that hold tokens < M
+            const int c_end = min(half, p.M - m_beg);
             for (int hs = 0; hs < kStrips; ++hs) {
                 const int n = (strip + hs) * kR + row;
-                const uint32_t tcol = tlane + 128u * hs;
-                auto put = [&](int c, uint32_t bits) {
-                    const int m = tt * p.BMT + c;
-                    if (n < p.N && m < p.M &&
-                        Q4_IN_BOUNDS(static_cast<long long>(m) * p.N + n, 1, static_cast<long long>(p.M) * p.N)) {
-                        float* dst = p.y + static_cast<long long>(m) * p.N + n;
-                        if (add)
-                            red_add_f32(dst, __uint_as_float(bits));
-                        else
-                            *dst = __uint_as_float(bits);
-                    }
-                };
-                int c0 = c_beg;
-                for (; c0 + 64 <= c_end; c0 += 64) {
-                    uint32_t v[64];
-                    tc_ld_x32(tcol + c0, v);
-                    tc_ld_x32(tcol + c0 + 32, v + 32);
-                    tc_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 64; ++i) put(c0 + i, v[i]);
-                }
-                for (; c0 + 32 <= c_end; c0 += 32) {
-                    uint32_t v[32];
-                    tc_ld_x32(tcol + c0, v);
-                    tc_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) put(c0 + i, v[i]);
-                }
-                for (; c0 < c_end; c0 += 8) {
+                const bool row_ok = n < p.N;
+                const uint32_t tcol = tlane + 128u * hs + static_cast<uint32_t>(wg * half);
+                float* dst0 = p.y + static_cast<long long>(m_beg) * p.N + n;
+#pragma unroll 1
+                for (int c0 = 0; c0 < c_end; c0 += 8) {
                     uint32_t v[8];
                     tc_ld_x8(tcol + c0, v);
                     tc_wait_ld();
+                    float* dst = dst0 + static_cast<long long>(c0) * p.N;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) put(c0 + i, v[i]);
+                    for (int i = 0; i < 8; ++i, dst += p.N) {
+                        if (!row_ok || c0 + i >= c_end ||
+                            !Q4_IN_BOUNDS(dst - p.y, 1, static_cast<long long>(p.M) * p.N))
+                            continue;
+                        if (add)
+                            red_add_f32(dst, __uint_as_float(v[i]));
+                        else
+                            *dst = __uint_as_float(v[i]);
+                    }
                 }
             }
             // the accumulator may now be overwritten by the next segment's MMAs
