@@ -14,8 +14,10 @@
 // which keeps every output inside 1e-4 * sum|W x| + 1e-6 with a margin of
 // ~0.3 sqrt(K) standard deviations (about 20 at K = 4096).
 //
-// Roles (one CTA per tile of 128 weight rows -- two strips of 128 when
-// BMT <= 128 -- x BMT tokens x one K chunk):
+// Work: a tile is 128 weight rows (two strips of 128 when BMT <= 128) x BMT
+// tokens.  CTAs are persistent, one per SM; each walks its list of segments
+// (a run of weight stages of one tile, see SegCursor), the rings below
+// running on from one segment to the next.  Roles:
 //  * warp 0 streams, by TMA, stages of 4 groups of codes (a 128-row x
 //    128-byte box, 128-byte swizzle) with their scales (cp.async);
 //  * warp 10 streams, by TMA, the x tile of every group (BMT tokens x 64 k
@@ -29,10 +31,12 @@
 //  * warp 1 owns the tensor memory and, per group, issues four tcgen05.mma
 //    M=128 N=BMT K=16 (A from tensor memory, B = x tile from shared memory)
 //    into one fp32 accumulator of BMT columns, then one commit that frees the
-//    group's ring slot (A slot and x stage together); a last commit marks the
-//    accumulator ready.
-//  * warps 2-9 then read the accumulator (tcgen05.ld) and write y, or add it
-//    into y with red.add when K is split across CTAs (y zeroed first).
+//    group's ring slot (A slot and x stage together); a commit at the end of
+//    a segment marks the accumulator ready, and the next segment's first
+//    MMA waits until the epilogue has read it out.
+//  * warps 2-9, at the start of each segment and after the last, read the
+//    previous segment's accumulator (tcgen05.ld) and store it into y (whole
+//    tiles) or add it with red.add (parts of a split tile; y zeroed first).
 // Measured on B200: with one thread issuing the MMAs, an x stream tied to the
 // weight stream and two commits per group, that thread spent most of each
 // group waiting for x and committing; the separate x warp and the shared
