@@ -29,6 +29,10 @@
 //  * Lane (g, tq) holds rows rho(g) and rho(g) + 8 of its warp's 16 with
 //    rho = (0 2 4 6 1 3 5 7): under the 128-byte swizzle the four rows a
 //    half-warp reads at once then fall in four different bank windows.
+//  * The scales of a stage (8 groups of a row, 16 bytes) arrive by cp.async
+//    two stages ahead, into the unused second half of the table's rows, when
+//    G is a multiple of 8 (scale rows in 16-byte blocks).  Loads one stage
+//    ahead into registers were the top stall (long scoreboard) at M = 8.
 //  * x of the CTA's K range is rounded to binary16 once into shared memory,
 //    token rows 16 bytes off a multiple of 32 (conflict-free B loads).
 //  * K is split across CTAs when x would not fit beside the ring, or when
@@ -97,6 +101,16 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     return v;
 }
 
+// A read of data another proxy or thread wrote: stays after the wait before it.
+__device__ __forceinline__ uint4 lds128_after_wait(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
 __device__ __forceinline__ uint32_t ldg_nc_u32(const void* p) {
     uint32_t v;
     asm("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
@@ -141,7 +155,21 @@ __device__ __forceinline__ float half_hi(uint32_t w) {
     return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
 }
 
-template <int MB, bool kEvenG>
+// Scales of a stage, copied ahead by cp.async into the unused second half of
+// the table's 256-byte rows: the 16 bytes (8 groups) of one weight row per
+// 16-byte slot; src_bytes < 16 zero-fills the rest (last stage, rows past N).
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+constexpr int kScDepth = 3;  // stages of scales in flight per warp
+
+// kAsyncSc (G a multiple of 8): scales come by cp.async two stages ahead into
+// shared memory; otherwise by loads one stage ahead into registers.
+template <int MB, bool kEvenG, bool kAsyncSc>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_small_kernel(const __grid_constant__ CUtensorMap cmap, const SmallP p) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -261,10 +289,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t xlane = base + kXOff + 32u * tq;
     bool bad = false;
 
-    // scales run one stage ahead: (nrb, ns) is the cursor of the next stage
+    // scales run ahead of the consumer: (nrb, ns) is the cursor of the next
+    // stage to fetch
     uint32_t sc_lo[4], sc_hi[4], nx_lo[4], nx_hi[4];
     int nrb = rb_first, ns = 0;
+    // kAsyncSc: warp w's slots are table rows 2 kScDepth w + 2 d + h, second
+    // half: stage d (mod kScDepth), rows r1 (h = 0) and r1 + 8 (h = 1), slot rho
+    const uint32_t sc_slots = base + static_cast<uint32_t>(2 * kScDepth * warp) * 256u + 128u +
+                              16u * static_cast<uint32_t>(rho);
+    int sc_issued = 0;
+    auto fetch_next = [&]() {
+        if (nrb < p.NB) {
+            if (tq == 0) {
+                const int g0 = (k0 + ns * kStageK) / kGroup;
+                const uint32_t bytes = static_cast<uint32_t>(min(8, p.G - g0)) * 2u;
+                const uint32_t d = static_cast<uint32_t>(sc_issued % kScDepth);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int row = nrb * kRows + r1 + 8 * h;
+                    const bool in = row < p.N &&
+                                    Q4_IN_BOUNDS(static_cast<int64_t>(row) * p.G + g0, bytes / 2,
+                                                 static_cast<int64_t>(p.N) * p.G);
+                    cp_async_16(sc_slots + (2u * d + h) * 256u,
+                                in ? p.scales + static_cast<int64_t>(row) * p.G + g0 : p.scales,
+                                in ? bytes : 0u);
+                }
+            }
+            if (++ns == nst) {
+                ns = 0;
+                nrb += p.rb_step;
+            }
+        }
+        ++sc_issued;
+        cp_async_commit();
+    };
     auto load_next = [&]() {
+        if (kAsyncSc) {
+            fetch_next();
+            return;
+        }
         if (nrb < p.NB) {
             int n1 = min(nrb * kRows + r1, p.N - 1), n2 = min(nrb * kRows + r1 + 8, p.N - 1);
             const int kb = k0 + ns * kStageK;
@@ -277,10 +340,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     };
+    if (kAsyncSc) fetch_next();  // two stages ahead: stages 0 and 1 now
     load_next();
 
     int slot = 0;
     uint32_t fparity = 0;
+    int sc_used = 0;
     for (int rb = rb_first; rb < p.NB; rb += p.rb_step) {
         float acc[MB][4];
 #pragma unroll
@@ -289,12 +354,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int q = 0; q < 4; ++q) acc[mb][q] = 0.f;
 
         for (int s = 0; s < nst; ++s) {
+            if (kAsyncSc) {
+                load_next();  // the stage two ahead
+                cp_async_wait<kScDepth - 1>();
+                __syncwarp();
+                const uint32_t d = static_cast<uint32_t>(sc_used % kScDepth);
+                const uint4 vl = lds128_after_wait(sc_slots + (2u * d) * 256u);
+                const uint4 vh = lds128_after_wait(sc_slots + (2u * d + 1u) * 256u);
+                sc_lo[0] = vl.x; sc_lo[1] = vl.y; sc_lo[2] = vl.z; sc_lo[3] = vl.w;
+                sc_hi[0] = vh.x; sc_hi[1] = vh.y; sc_hi[2] = vh.z; sc_hi[3] = vh.w;
+                ++sc_used;
+            } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                sc_lo[i] = nx_lo[i];
-                sc_hi[i] = nx_hi[i];
+                for (int i = 0; i < 4; ++i) {
+                    sc_lo[i] = nx_lo[i];
+                    sc_hi[i] = nx_hi[i];
+                }
+                load_next();
             }
-            load_next();
             const int kb = k0 + s * kStageK;
             if (!bad && !mbar_wait(bars + 8u * slot, fparity)) {
                 bad = true;
@@ -400,12 +477,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
     }
+    if (kAsyncSc) cp_async_wait<0>();  // no copy outlives the block
 }
 
-template <int MB, bool kEvenG>
+template <int MB, bool kEvenG, bool kAsyncSc = false>
 cudaError_t launch_variant(const CUtensorMap& cmap, const SmallP& p, int grid, int smem, int slot,
                            cudaStream_t s, const DeviceInfo& dev) {
-    auto kern = gemm_small_kernel<MB, kEvenG>;
+    auto kern = gemm_small_kernel<MB, kEvenG, kAsyncSc>;
     cudaError_t e = ensure_smem_attr(reinterpret_cast<const void*>(kern), smem, slot, dev.device);
     if (e != cudaSuccess) return e;
     kern<<<grid, kThreads, smem, s>>>(cmap, p);
@@ -479,6 +557,12 @@ cudaError_t launch_gemm_small(const uint8_t* codes, const uint16_t* scales, cons
         if (e != cudaSuccess) return e;
     }
     const bool even = (p.G & 1) == 0;
+    if (p.G % 8 == 0) {  // scale rows in 16-byte blocks: cp.async ahead
+        if (M <= 8) return launch_variant<1, true, true>(cmap, p, best_grid, smem, 70, s, dev);
+        if (M <= 16) return launch_variant<2, true, true>(cmap, p, best_grid, smem, 71, s, dev);
+        if (M <= 24) return launch_variant<3, true, true>(cmap, p, best_grid, smem, 72, s, dev);
+        return launch_variant<4, true, true>(cmap, p, best_grid, smem, 73, s, dev);
+    }
     if (M <= 8)
         return even ? launch_variant<1, true>(cmap, p, best_grid, smem, 40, s, dev)
                     : launch_variant<1, false>(cmap, p, best_grid, smem, 41, s, dev);
