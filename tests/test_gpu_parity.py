@@ -457,6 +457,29 @@ def test_llama2_70b_prefill(linear, M):
     assert ok, f"{linear} M={M}: worst err/bound = {worst:.3g}"
 
 
+@pytest.mark.parametrize("M,N,K", [
+    (300, 40000, 128),   # one weight stage per tile, 626 whole tiles dealt over 148 CTAs
+    (256, 19200, 512),   # stream-K: one whole tile per CTA, then 2 leftover tiles shared out
+    (40, 38000, 64),     # two-strip tiles, a single group per tile, 149 tiles on 148 CTAs
+    (130, 2000, 4160),   # odd G (65), two token tiles of 65: K in 6 chunks, plain scale loads
+    (256, 10240, 8256),  # odd G (129) under stream-K with no whole tiles
+])
+def test_tensor_core_plans(M, N, K):
+    """The persistent tensor-core kernel's plans at their edges (whole tiles,
+    stream-K leftovers, chunks, one-stage tiles, odd group counts): every
+    token x the first and last row of every 128-row strip plus 512 seeded
+    random rows, against the oracle."""
+    codes, scales = synth.tiny_codes_scales(900 + M, N, K)
+    x = synth.activations(901 + M, M, K)
+    y = run_matmul(codes, scales, NF4, x)
+    assert np.all(np.isfinite(y))
+    rows = strip_rows(N, M + 7, n_random=512)
+    y_ref, a = oracle_matmul_parallel(codes, scales, NF4, x, rows=rows)
+    ok, worst = within_tolerance(y[:, rows], y_ref, a)
+    assert ok, f"M={M} N={N} K={K}: worst err/bound = {worst:.3g}"
+    assert q4.timeout_flags() == 0
+
+
 def test_tensor_core_path_allocates_nothing():
     """q4_gemm at M > 24 keeps the binary16 copy of x in the library's fixed
     array: after a warm-up call has loaded the kernels, a call whose copy of x

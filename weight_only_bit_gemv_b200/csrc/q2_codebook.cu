@@ -448,11 +448,14 @@ __device__ __forceinline__ void copy_scales(uint32_t dst, const uint16_t* src) {
 
 // kWhole: a tile is one stage (rows of at most 2 KB); kSW: bytes per scale
 // copy (16, 8, 4 with cp.async; 2 = plain loads, for an odd group count).
-// kLut: word quarters q = 0, 1 of every group are decoded through a per-lane
-// byte -> four binary16 values table in shared memory (one LDS.64 and one PRMT
-// per four weights) instead of by PRMT from the codebook registers (about 2.4
-// ALU instructions per weight), which moves half of the decode from the ALU
-// pipe to the shared-memory pipe.
+// kLut: the word quarters q < kR2LutQuarters of every group are decoded
+// through a per-lane byte -> four binary16 values table in shared memory (one
+// LDS.64 and one PRMT per four weights) instead of by PRMT from the codebook
+// registers (about 2.4 ALU instructions per weight), which moves the decode
+// from the ALU pipe to the shared-memory pipe.  Measured on B200 (70B
+// linears): table for 2 quarters 63.9 us on gate_up, 3: 62.3, 4: 61.4.
+constexpr int kR2LutQuarters = 4;  // quarters decoded through the table when kLut
+
 template <bool kWhole, int kSW, bool kLut>
 __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -604,7 +607,7 @@ __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
                 v1 = __ldg(src + 1);
             }
             const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            const bool by_table = kLut && q < 2;
+            const bool by_table = kLut && q < kR2LutQuarters;
 #pragma unroll
             for (int mm = 0; mm < 8; ++mm) {
                 const int i = mm >> 1, h = mm & 1, m = 8 * q + mm;
@@ -666,7 +669,7 @@ __global__ void __launch_bounds__(kR2Threads, 1) gemv2_ring_kernel(const G2 p) {
                         const uint32_t xb1[8] = {xw0.x, xw0.y, xw0.z, xw0.w, xw1.x, xw1.y, xw1.z, xw1.w};
                         const uint32_t wlg = word4(lo_g, q), whg = word4(hi_g, q);
                         const uint32_t wlh = word4(lo_h, q), whh = word4(hi_h, q);
-                        if (kLut && q < 2) {
+                        if (kLut && q < kR2LutQuarters) {
                             const uint32_t lane8 = static_cast<uint32_t>(lane) * 8u;
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
