@@ -58,8 +58,8 @@ def peaks():
 # (4096 -> 22016) from an ncu capture, with the SHA-1 of the kernel source it
 # was taken on; when the source changes the figure no longer applies and the
 # bench reports null.
-GEMV_TRAFFIC = {"bytes": 47953152 + 0,
-                "source_sha1": "dedcf912d557a0e31a9d3a1eb0f8526aac59428a",
+GEMV_TRAFFIC = {"bytes": 47952896,
+                "source_sha1": "96e7038247d1cef1a06a1c422a6ee1555db83a0f",
                 "capture": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum "
                            "--clock-control none -k regex:gemv_m1 -s 2 -c 1 python -m "
                            "weight_only_bit_gemv_b200.profile_case --workload llama2_7b_layer "
