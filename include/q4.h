@@ -168,8 +168,10 @@ q4_status q4_gemv(const uint8_t* codes, const uint16_t* scales,
  * x is rounded to binary16, and products accumulate in binary32 in tensor
  * memory.  Either way the result is within 1e-4 * sum_k |W x| + 1e-6 of the
  * exact sum per element (for the tensor-core path this holds statistically:
- * the binary16 rounding of W and x is a relative error of at most 2^-11 per
- * term, far inside the bound once K is a few hundred).
+ * the binary16 rounding of W is a relative error of at most 2^-11 per term,
+ * which sums to about 1/(0.32 sqrt(K)) of the bound per standard deviation:
+ * 20 at K = 4096, 7 at K = 512, but at K = 128 a few outputs in a million
+ * can exceed the bound).
  * The tensor-core path first converts x to binary16 into a fixed 32 MiB
  * device array (see Ownership), in chunks of tokens when 2 * M * K is
  * larger.  Calls that take this path are ordered through one event per
@@ -177,10 +179,12 @@ q4_status q4_gemv(const uint8_t* codes, const uint16_t* scales,
  * at the same time (they may serialize on the GPU); under stream capture the
  * ordering becomes external event nodes of the graph.  The first such call on
  * a device looks up the array's address and creates the event: make it
- * before any stream capture (q4_step_create does this itself).  When the
- * K dimension is split across thread blocks, y is zeroed on the stream and
- * the partial sums are added into it atomically, so the summation order (and
- * the last bits of y) may vary between runs.
+ * before any stream capture (q4_step_create does this itself).  The
+ * tensor-core kernel runs one persistent block per SM; where a tile's K range
+ * is shared between blocks, that tile's y is zeroed first (by the x
+ * conversion or a memset on the stream) and the partial sums are added into
+ * it atomically, so the summation order (and the last bits of y) may vary
+ * between runs.
  * In: codes, scales, codebook, x [M][K] bf16.  Out: y [M][N] fp32.
  */
 q4_status q4_gemm(const uint8_t* codes, const uint16_t* scales,
