@@ -23,8 +23,8 @@ pytestmark = pytest.mark.gpu
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 # every kernel family on ragged and edge shapes: M = 1 rings, M = 2..24,
-# tensor cores (chunked too), two-bit, pack / dequant / embed, the
-# allocation-free entry point and a recorded step
+# tensor cores (chunked, and every kind of persistent plan), two-bit, pack /
+# dequant / embed, the allocation-free entry point and a recorded step
 SELECTION = [
     "tests/test_gpu_parity.py::test_ragged_shapes",
     "tests/test_gpu_parity.py::test_gemv2_ragged",
@@ -37,6 +37,7 @@ SELECTION = [
     "tests/test_gpu_parity.py::test_gemv2_output_bounds_and_stream",
     "tests/test_gpu_parity.py::test_integer_codebook_exact",
     "tests/test_gpu_parity.py::test_tensor_core_path_chunks_large_inputs",
+    "tests/test_gpu_parity.py::test_tensor_core_plans",
     "tests/test_gpu_step.py::test_step_replays_every_path",
     "tests/test_zz_no_alloc.py",
 ]
